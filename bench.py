@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the chunked H2O step (prefill of one synthetic sequence).
+
+A bench step is one prefill of the workload's whole sequence: the cache is
+reset and all N/T chunks go through ``h2o_step`` (for the default workload
+64 chunks of 1024 tokens against a 2048-slot cache, Qwen3-4B layer shape).
+All chunks' inputs are resident in HBM before timing (they exceed the L2
+cache, so no flush is needed). ``value`` is tokens/s over all ranks; each
+rank runs its own sequence (weak scaling, no collective on the data path).
+
+Also reported: per-kernel device times from CUDA events inside the step
+(roofline of the dominant kernel), the end-to-end number through
+``h2o_step_host`` with pinned host buffers, SM clocks sampled during the
+timed region, and the fp64 oracle timed on a bounded sample on the host
+cores (``cpu_baseline``). ``--impl reference`` times the oracle alone.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from h2o_kv_cache_step_b200 import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "qwen3-4b-c2048-t1024-n64k"
+METRIC = "H2O prefill tokens/sec per layer (C=2048,T=1024,64k) + % bf16 tensor peak"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ---------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, flag in zip(names, parts[5:9]):
+                if flag.lower() in ("active", "1"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------- algorithmic work ---
+def step_pairs(wl, n: int, T: int) -> int:
+    """Visible (query row, key) pairs of one chunk step with n valid slots."""
+    return wl.B * wl.Hq * (T * n + T * (T + 1) // 2)
+
+
+def sequence_schedule(wl):
+    """(n before the step, T) for every chunk of one sequence prefill."""
+    out, n = [], 0
+    for _ in range(wl.n_chunks):
+        out.append((n, wl.T))
+        n = min(wl.C, n + wl.T)
+    return out
+
+
+def kernel_work(wl, name: str, n: int, T: int):
+    """Algorithmic work of one launch: (amount, unit, bound)."""
+    pairs = step_pairs(wl, n, T)
+    if "sdpa" in name:
+        return 4.0 * wl.d * pairs, "flop", "tensor"      # QK^T + PV
+    if "wsum" in name:
+        return 2.0 * wl.d * pairs, "flop", "tensor"      # QK^T recompute
+    e = 2 if wl.dtype == "bf16" else 4
+    groups = wl.B * wl.Hkv
+    if "select" in name:
+        return float(groups * (n + T) * 9 + groups * wl.C * 8), "byte", "hbm"
+    if "scatter" in name:
+        kept = min(T, wl.C)
+        return float(groups * kept * wl.d * e * 4), "byte", "hbm"  # read+write K and V rows
+    return 0.0, "byte", "hbm"
+
+
+# ------------------------------------------------------------------ ours ---
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from h2o_kv_cache_step_b200 import H2OCache
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synth.WORKLOADS[args.workload]
+    if world > 1:
+        wl = wl.with_(seed=wl.seed + 1000 * rank)  # each rank prefills its own sequence
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    sched = sequence_schedule(wl)
+
+    t0 = time.time()
+    chunks = []
+    for c in range(wl.n_chunks):
+        q, k, v = synth.chunk(wl, c)
+        chunks.append(tuple(torch.from_numpy(x).to(dev).to(tdt) for x in (q, k, v)))
+    torch.cuda.synchronize()
+    in_bytes = sum(t.numel() * t.element_size() for ch in chunks for t in ch)
+    log(f"[rank {rank}] generated {wl.n_chunks} chunks ({in_bytes / 1e6:.0f} MB resident) "
+        f"in {time.time() - t0:.1f}s")
+    out = torch.empty_like(chunks[0][0])
+    cache = H2OCache(wl.B, wl.Hq, wl.Hkv, wl.d, wl.C, tdt, max_T=wl.T)
+    plan = cache.kernel_plan(wl.T)
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        cache.reset()
+        for (q, k, v) in chunks:
+            cache.step(q, k, v, out=out)
+
+    for _ in range(args.warmup):
+        prefill()
+    cache.sync_check()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    cache.profile_begin(args.steps * wl.n_chunks)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        prefill()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    prof = cache.profile_end()
+    clk = clocks.stop() if clocks else None
+    cache.sync_check()
+
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_per_step = ms_total / args.steps
+    tokens = wl.B * wl.N * args.steps * world
+    value = tokens / (ms_total / 1e3)
+
+    # roofline of the dominant kernel
+    peaks, peak_kind = measured_peaks()
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
+    roof = None
+    kernels = {}
+    for name, (ms, cnt) in prof.items():
+        work = sum(kernel_work(wl, name, n, T)[0] for (n, T) in sched) * args.steps
+        _, unit, bound = kernel_work(wl, name, 0, wl.T)
+        avg_ms = ms / max(cnt, 1)
+        work_per_launch = work / max(cnt, 1)
+        kernels[name] = {"launches": cnt, "ms_total": round(ms, 4), "share": round(ms / sum(
+            v[0] for v in prof.values()), 4), "avg_us": round(avg_ms * 1e3, 2)}
+        if unit == "flop":
+            kernels[name]["tflops"] = round(work_per_launch / (avg_ms * 1e-3) / 1e12, 1)
+        else:
+            kernels[name]["gbs"] = round(work_per_launch / (avg_ms * 1e-3) / 1e9, 1)
+    if dom:
+        ms, cnt = prof[dom]
+        work = sum(kernel_work(wl, dom, n, T)[0] for (n, T) in sched) * args.steps
+        _, unit, bound = kernel_work(wl, dom, 0, wl.T)
+        per_launch = work / cnt
+        avg_s = ms / cnt * 1e-3
+        if unit == "flop":
+            achieved = per_launch / avg_s / 1e12
+            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "traffic": None,
+                    "peak_source": f"{peak_kind} bf16 sustained (kernel timed inside a long step)",
+                    "work_per_launch": per_launch}
+        else:
+            achieved = per_launch / avg_s / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                    "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                    "peak_source": f"{peak_kind} HBM copy", "work_per_launch": per_launch}
+    # tensor-core fraction of the whole fused SDPA + weight-sum path (6d count)
+    path_flops = sum(6.0 * wl.d * step_pairs(wl, n, T) for (n, T) in sched) * args.steps
+    path_ms = sum(ms for name, (ms, _) in prof.items() if ("sdpa" in name or "wsum" in name))
+    fused = None
+    if path_ms > 0:
+        ach = path_flops / (path_ms * 1e-3) / 1e12
+        fused = {"achieved_tflops": round(ach, 1),
+                 "frac_of_measured_burst": round(ach / peaks["bf16_tflops"], 4),
+                 "frac_of_spec_2250": round(ach / 2250.0, 4)}
+
+    # end to end through h2o_step_host with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = [tuple(t.cpu().pin_memory() for t in ch) for ch in chunks]
+        hout = torch.empty_like(chunks[0][0], device="cpu").pin_memory()
+        h2d = sum(t.numel() * t.element_size() for ch in host for t in ch)
+        d2h = hout.numel() * hout.element_size() * wl.n_chunks
+        cache.reset()
+        for (q, k, v) in host[:2]:
+            cache.step_host(q, k, v, hout)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        reps = max(1, min(args.steps, 3))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            cache.reset()
+            for (q, k, v) in host:
+                cache.step_host(q, k, v, hout)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": round(wl.B * wl.N * reps * world / (ems / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "h2o_step_host (pinned host buffers, synchronous per chunk)"}
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.dtype,
+        "data": "synthetic (seeded; Qwen3-4B-shaped layer, heavy-hitter keys)",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                   "C": wl.C, "T": wl.T, "N": wl.N, "chunks_per_step": wl.n_chunks,
+                   "global_batch": wl.B * world, "seq_len": wl.N, "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB resident per rank)"},
+        "gpu_launches": sum(cnt for (_, cnt) in prof.values()),
+        "kernel_plan": plan,
+        "kernels": kernels,
+        "roofline": roof,
+        "fused_sdpa_wsum_6d": fused,
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    cache.close()
+    return result, wl
+
+
+# ---------------------------------------------------------- oracle (CPU) ---
+def oracle_sample(wl, groups_wanted: int):
+    """Time the fp64 oracle on one steady-state chunk step of `groups_wanted`
+    (batch, KV head) groups (OpenMP over groups); returns seconds, groups,
+    threads."""
+    from oracle import oracle
+    threads = os.cpu_count() or 1
+    c = min(wl.n_chunks - 1, wl.C // wl.T + 1)  # first chunk with a full cache
+    P = c * wl.T
+    q, k, v = synth.chunk(wl, c)
+    K, V, S, pos = synth.random_state(wl, n=wl.C, P=P, seed=1)
+    G = wl.G
+    g_total = wl.B * wl.Hkv
+    ng = max(1, min(groups_wanted, g_total))
+    # the first ng groups (b-major), as a batch of single-group problems
+    sel = [(b, g) for b in range(wl.B) for g in range(wl.Hkv)][:ng]
+    Ks = np.stack([K[b, g] for b, g in sel])[:, None].astype(np.float64)
+    Vs = np.stack([V[b, g] for b, g in sel])[:, None].astype(np.float64)
+    Ss = np.stack([S[b, g] for b, g in sel])[:, None].astype(np.float64)
+    Ps = np.stack([pos[b, g] for b, g in sel])[:, None].astype(np.int64)
+    qs = np.stack([q[b, g * G:(g + 1) * G] for b, g in sel]).astype(np.float64)
+    ks = np.stack([k[b, g] for b, g in sel])[:, None].astype(np.float64)
+    vs = np.stack([v[b, g] for b, g in sel])[:, None].astype(np.float64)
+    # batch dim = ng, one KV head each, G query heads each
+    st = oracle.State(Ks, Vs, Ss, Ps, P)
+    t0 = time.perf_counter()
+    oracle.step(st, qs, ks, vs, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return dt, ng, min(threads, ng)
+
+
+def cpu_baseline_line(wl, groups_wanted):
+    dt, ng, thr = oracle_sample(wl, groups_wanted)
+    g_total = wl.B * wl.Hkv
+    # steady-state step time extrapolated to all groups at this thread count
+    step_s = dt * (g_total / ng)
+    tok_s = wl.B * wl.T / step_s
+    return {"value": round(tok_s, 2), "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": (f"one steady-state chunk step (n=C={wl.C}, T={wl.T}) of {ng} of {g_total} "
+                       f"KV groups in {dt:.2f}s, fp64 C oracle, OpenMP over groups; "
+                       f"extrapolated to all groups")}
+
+
+def run_reference(args):
+    wl = synth.WORKLOADS[args.workload]
+    groups = min(os.cpu_count() or 1, wl.B * wl.Hkv)
+    from oracle import oracle
+    oracle.build()
+    for _ in range(args.warmup):
+        oracle_sample(wl, groups)
+    times = []
+    ng = thr = 0
+    for _ in range(args.steps):
+        dt, ng, thr = oracle_sample(wl, groups)
+        times.append(dt * (wl.B * wl.Hkv) / ng)
+    step_s = float(np.mean(times))
+    # a bench step is a whole-sequence prefill: extrapolate the steady-state
+    # chunk time over the sequence's chunks (fill chunks cost less; this
+    # overstates the oracle's time slightly)
+    seq_s = step_s * wl.n_chunks
+    value = wl.B * wl.N / seq_s
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(seq_s * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                       "C": wl.C, "T": wl.T, "N": wl.N},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": thr,
+                             "kind": "oracle",
+                             "sample": f"per step: one steady-state chunk of {ng} of "
+                                       f"{wl.B * wl.Hkv} KV groups, extrapolated to the "
+                                       f"{wl.n_chunks}-chunk sequence"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-groups", type=int, default=0,
+                    help="KV groups in the oracle sample (default: host cores)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        log("warning: fewer than 3 warm-up steps")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    result, wl = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            groups = args.cpu_groups or min(os.cpu_count() or 1, wl.B * wl.Hkv)
+            result["cpu_baseline"] = cpu_baseline_line(synth.WORKLOADS[args.workload], groups)
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,610 @@
+// h2o.cu -- the C ABI of the chunked H2O step (declared in include/h2o.h).
+//
+// Owns the context: the cache (keys, values, H2O scores, positions) for every
+// (sequence, KV head), the per-step workspace and the device error word; and
+// issues one step as a fixed, stream-ordered sequence of kernels:
+//   1. chunk SDPA, writing the output and each row's log-sum-exp;
+//   2. per-key attention-weight sums, added to the H2O scores;
+//   3. selection of the C survivors and the token -> slot map;
+//   4. copy of the surviving chunk keys/values into their slots.
+// No step of the path runs on the host: the host validates arguments, keeps
+// the two counters (P, n) and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/h2o.h"
+#include "kernels.h"
+#include "tc.h"
+
+using namespace h2o;
+
+namespace {
+
+thread_local char g_thread_err[512] = "";
+
+void set_thread_err(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_thread_err, sizeof(g_thread_err), fmt, ap);
+    va_end(ap);
+}
+
+}  // namespace
+
+struct h2o_ctx {
+    int B, Hq, Hkv, d, C, dtype, tmax;
+    int device;
+    int num_sms;
+    int64_t P, n;
+    size_t elem;
+    // cache
+    void* Kc = nullptr;
+    void* Vc = nullptr;
+    float* scores = nullptr;
+    int32_t* pos = nullptr;
+    // workspace (capacity tmax tokens)
+    float* lse = nullptr;
+    float* cand_score = nullptr;
+    int32_t* cand_pos = nullptr;
+    uint8_t* cand_kept = nullptr;
+    int32_t* token_slot = nullptr;
+    int32_t* free_list = nullptr;
+    float* partials = nullptr;
+    size_t partial_elems = 0;
+    // host staging for h2o_step_host
+    void* stage = nullptr;
+    size_t stage_bytes = 0;
+    // error word (host-mapped)
+    int* err_host = nullptr;
+    int* err_dev = nullptr;
+    unsigned long long wait_ns;
+    int poisoned = 0;
+    // last step
+    int last_T = 0, last_n = 0;
+    bool use_tc = false;
+    // per-kernel profiling
+    bool prof_on = false;
+    int prof_max_steps = 0, prof_steps = 0;
+    std::vector<cudaEvent_t> prof_ev;      // (kMaxStepKernels + 1) per step
+    std::vector<LaunchLog> prof_logs;
+    char err[512];
+};
+
+namespace {
+
+int fail(h2o_ctx* c, int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    if (c) {
+        snprintf(c->err, sizeof(c->err), "%s", buf);
+    } else {
+        snprintf(g_thread_err, sizeof(g_thread_err), "%s", buf);
+    }
+    return code;
+}
+
+int cuda_fail(h2o_ctx* c, cudaError_t e, const char* what) {
+    return fail(c, e == cudaErrorMemoryAllocation ? H2O_ERR_OOM : H2O_ERR_CUDA, "%s: %s (%s)", what,
+                cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+#define H2O_TRY(ctx, expr, what)                        \
+    do {                                                \
+        cudaError_t e_ = (expr);                        \
+        if (e_ != cudaSuccess) return cuda_fail(ctx, e_, what); \
+    } while (0)
+
+// Makes the context's device current for the lifetime of the object.
+struct DeviceGuard {
+    int prev = -1;
+    bool changed = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+            changed = cudaSetDevice(dev) == cudaSuccess;
+        }
+    }
+    ~DeviceGuard() {
+        if (changed) cudaSetDevice(prev);
+    }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void free_workspace(h2o_ctx* c) {
+    cudaFree(c->lse);
+    cudaFree(c->cand_score);
+    cudaFree(c->cand_pos);
+    cudaFree(c->cand_kept);
+    cudaFree(c->token_slot);
+    cudaFree(c->partials);
+    c->lse = c->cand_score = c->partials = nullptr;
+    c->cand_pos = c->token_slot = nullptr;
+    c->cand_kept = nullptr;
+    c->partial_elems = 0;
+}
+
+int alloc_workspace(h2o_ctx* c, int tmax) {
+    const size_t groups = (size_t)c->B * c->Hkv;
+    const size_t cs = (size_t)c->C + tmax;
+    H2O_TRY(c, cudaMalloc(&c->lse, sizeof(float) * (size_t)c->B * c->Hq * tmax), "cudaMalloc(lse)");
+    H2O_TRY(c, cudaMalloc(&c->cand_score, sizeof(float) * groups * cs), "cudaMalloc(cand_score)");
+    H2O_TRY(c, cudaMalloc(&c->cand_pos, sizeof(int32_t) * groups * cs), "cudaMalloc(cand_pos)");
+    H2O_TRY(c, cudaMalloc(&c->cand_kept, groups * cs), "cudaMalloc(cand_kept)");
+    H2O_TRY(c, cudaMalloc(&c->token_slot, sizeof(int32_t) * groups * tmax), "cudaMalloc(token_slot)");
+    c->partial_elems = tc_partial_elems(c->B, c->Hq, c->Hkv, c->C, tmax);
+    if (c->partial_elems)
+        H2O_TRY(c, cudaMalloc(&c->partials, sizeof(float) * c->partial_elems), "cudaMalloc(partials)");
+    c->tmax = tmax;
+    return H2O_OK;
+}
+
+int check_ctx(h2o_ctx* c) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    if (c->poisoned) return fail(c, H2O_ERR_POISONED, "context poisoned by an earlier device error");
+    const int word = *(volatile int*)c->err_host;
+    if (word != kDevOk) {
+        c->poisoned = 1;
+        return fail(c, H2O_ERR_TIMEOUT, "a kernel stopped after a bounded wait ran out (device code %d)",
+                    word);
+    }
+    return H2O_OK;
+}
+
+StepArgs make_args(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T,
+                   cudaStream_t s) {
+    StepArgs a{};
+    a.B = c->B;
+    a.Hq = c->Hq;
+    a.Hkv = c->Hkv;
+    a.d = c->d;
+    a.C = c->C;
+    a.T = T;
+    a.n = (int)c->n;
+    a.P = c->P;
+    a.dtype = c->dtype;
+    a.tmax = c->tmax;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.out = out;
+    a.Kc = c->Kc;
+    a.Vc = c->Vc;
+    a.scores = c->scores;
+    a.pos = c->pos;
+    a.lse = c->lse;
+    a.cand_score = c->cand_score;
+    a.cand_pos = c->cand_pos;
+    a.cand_kept = c->cand_kept;
+    a.token_slot = c->token_slot;
+    a.free_list = c->free_list;
+    a.partials = c->partials;
+    a.partial_elems = c->partial_elems;
+    a.wb.err_word = c->err_dev;
+    a.wb.ns = c->wait_ns;
+    a.stream = s;
+    a.num_sms = c->num_sms;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* h2o_version(void) { return "h2o_kv_cache_step_b200 0.1 (sm_100a)"; }
+
+const char* h2o_last_error(const h2o_ctx* c) { return c ? c->err : g_thread_err; }
+
+int h2o_create_ex(int B, int Hq, int Hkv, int d, int C, int dtype, int max_T, h2o_ctx** out) {
+    if (!out) return fail(nullptr, H2O_ERR_ARG, "out is NULL");
+    *out = nullptr;
+    if (B < 1 || Hq < 1 || Hkv < 1 || C < 1 || max_T < 1)
+        return fail(nullptr, H2O_ERR_ARG, "B, Hq, Hkv, C, max_T must be >= 1");
+    if (Hq % Hkv != 0) return fail(nullptr, H2O_ERR_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (d != 64 && d != 128) return fail(nullptr, H2O_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+    if (dtype != H2O_BF16 && dtype != H2O_FP32) return fail(nullptr, H2O_ERR_ARG, "unknown dtype %d", dtype);
+    if ((long long)C + max_T > (1ll << 30)) return fail(nullptr, H2O_ERR_UNSUPPORTED, "C + max_T too large");
+
+    h2o_ctx* c = new (std::nothrow) h2o_ctx();
+    if (!c) return fail(nullptr, H2O_ERR_OOM, "host allocation failed");
+    c->B = B;
+    c->Hq = Hq;
+    c->Hkv = Hkv;
+    c->d = d;
+    c->C = C;
+    c->dtype = dtype;
+    c->elem = dtype == H2O_FP32 ? 4 : 2;
+    c->P = 0;
+    c->n = 0;
+    c->err[0] = 0;
+    const char* env = getenv("H2O_WAIT_TIMEOUT_MS");
+    long long ms = env ? atoll(env) : 0;
+    c->wait_ns = (unsigned long long)(ms > 0 ? ms : 2000) * 1000000ull;
+
+    auto bail = [&](int rc) {
+        snprintf(g_thread_err, sizeof(g_thread_err), "%s", c->err);
+        h2o_destroy(c);
+        return rc;
+    };
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e != cudaSuccess) return bail(cuda_fail(c, e, "cudaGetDevice"));
+    e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+    if (e != cudaSuccess) return bail(cuda_fail(c, e, "cudaDeviceGetAttribute"));
+    const size_t groups = (size_t)B * Hkv;
+    const size_t cache_bytes = groups * C * d * c->elem;
+    if ((e = cudaMalloc(&c->Kc, cache_bytes)) != cudaSuccess) return bail(cuda_fail(c, e, "cudaMalloc(K cache)"));
+    if ((e = cudaMalloc(&c->Vc, cache_bytes)) != cudaSuccess) return bail(cuda_fail(c, e, "cudaMalloc(V cache)"));
+    if ((e = cudaMalloc(&c->scores, sizeof(float) * groups * C)) != cudaSuccess)
+        return bail(cuda_fail(c, e, "cudaMalloc(scores)"));
+    if ((e = cudaMalloc(&c->pos, sizeof(int32_t) * groups * C)) != cudaSuccess)
+        return bail(cuda_fail(c, e, "cudaMalloc(positions)"));
+    if ((e = cudaMalloc(&c->free_list, sizeof(int32_t) * groups * C)) != cudaSuccess)
+        return bail(cuda_fail(c, e, "cudaMalloc(free_list)"));
+    int rc = alloc_workspace(c, max_T);
+    if (rc != H2O_OK) return bail(rc);
+    if ((e = cudaHostAlloc((void**)&c->err_host, sizeof(int), cudaHostAllocMapped)) != cudaSuccess)
+        return bail(cuda_fail(c, e, "cudaHostAlloc(error word)"));
+    *c->err_host = kDevOk;
+    if ((e = cudaHostGetDevicePointer((void**)&c->err_dev, c->err_host, 0)) != cudaSuccess)
+        return bail(cuda_fail(c, e, "cudaHostGetDevicePointer(error word)"));
+    c->use_tc = (dtype == H2O_BF16) && tc_supported(c->device, d);
+    rc = h2o_reset(c, nullptr);
+    if (rc != H2O_OK) return bail(rc);
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(cuda_fail(c, e, "initial clear"));
+    *out = c;
+    return H2O_OK;
+}
+
+int h2o_create(int B, int Hq, int Hkv, int d, int C, h2o_ctx** out) {
+    return h2o_create_ex(B, Hq, Hkv, d, C, H2O_BF16, C, out);
+}
+
+int h2o_destroy(h2o_ctx* c) {
+    if (!c) return H2O_OK;
+    DeviceGuard g(c->device);
+    cudaDeviceSynchronize();
+    free_workspace(c);
+    for (cudaEvent_t e : c->prof_ev) cudaEventDestroy(e);
+    cudaFree(c->Kc);
+    cudaFree(c->Vc);
+    cudaFree(c->scores);
+    cudaFree(c->pos);
+    cudaFree(c->free_list);
+    cudaFree(c->stage);
+    if (c->err_host) cudaFreeHost(c->err_host);
+    delete c;
+    return H2O_OK;
+}
+
+int h2o_reset(h2o_ctx* c, void* stream) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t groups = (size_t)c->B * c->Hkv;
+    H2O_TRY(c, cudaMemsetAsync(c->scores, 0, sizeof(float) * groups * c->C, s), "reset scores");
+    H2O_TRY(c, cudaMemsetAsync(c->pos, 0xff, sizeof(int32_t) * groups * c->C, s), "reset positions");
+    H2O_TRY(c, cudaMemsetAsync(c->Kc, 0, groups * c->C * c->d * c->elem, s), "reset K");
+    H2O_TRY(c, cudaMemsetAsync(c->Vc, 0, groups * c->C * c->d * c->elem, s), "reset V");
+    c->P = 0;
+    c->n = 0;
+    c->last_T = 0;
+    c->last_n = 0;
+    return H2O_OK;
+}
+
+int h2o_kernel_plan(const h2o_ctx* c, int T, const char** names, int max_names) {
+    if (!c || T < 1) return fail(nullptr, H2O_ERR_ARG, "bad arguments");
+    const char* plan[kMaxStepKernels];
+    int k = 0;
+    if (c->use_tc) {
+        k = tc_kernel_plan(c->B, c->Hq, c->Hkv, c->d, c->C, T, (int)c->n, plan, kMaxStepKernels - 2);
+    } else {
+        plan[k++] = "sdpa_simt_kernel";
+        plan[k++] = "wsum_simt_kernel";
+    }
+    plan[k++] = "select_kernel";
+    plan[k++] = "scatter_kernel";
+    for (int i = 0; i < k && i < max_names; ++i)
+        if (names) names[i] = plan[i];
+    return k;
+}
+
+int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (T < 1) return fail(c, H2O_ERR_ARG, "T must be >= 1 (got %d)", T);
+    if (!q || !k || !v || !out) return fail(c, H2O_ERR_ARG, "q, k, v, out must be non-NULL");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(c, H2O_ERR_ALIGN, "q, k, v, out must be 16-byte aligned");
+    if (c->P + T > (int64_t)INT32_MAX) return fail(c, H2O_ERR_UNSUPPORTED, "positions would exceed 2^31-1");
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T > c->tmax) {
+        H2O_TRY(c, cudaStreamSynchronize(s), "sync before workspace growth");
+        H2O_TRY(c, cudaDeviceSynchronize(), "sync before workspace growth");
+        free_workspace(c);
+        rc = alloc_workspace(c, T);
+        if (rc != H2O_OK) return rc;
+    }
+    StepArgs a = make_args(c, q, k, v, out, T, s);
+    LaunchLog local_log;
+    a.log = &local_log;
+    if (c->prof_on && c->prof_steps < c->prof_max_steps) {
+        const int slot = c->prof_steps++;
+        a.log = &c->prof_logs[slot];
+        a.log->n = 0;
+        a.log->ev = &c->prof_ev[(size_t)slot * (kMaxStepKernels + 1)];
+        H2O_TRY(c, cudaEventRecord(a.log->ev[0], s), "record profiling event");
+    }
+    if (c->use_tc) {
+        H2O_TRY(c, tc_sdpa(a), "launch tensor-core SDPA");
+        H2O_TRY(c, tc_wsum(a), "launch tensor-core weight sums");
+    } else {
+        H2O_TRY(c, launch_sdpa_simt(a), "launch SDPA");
+        H2O_TRY(c, launch_wsum_simt(a), "launch weight sums");
+    }
+    H2O_TRY(c, launch_select(a), "launch select");
+    H2O_TRY(c, launch_scatter(a), "launch scatter");
+    c->last_T = T;
+    c->last_n = (int)c->n;
+    c->n = std::min<int64_t>(c->C, c->n + T);
+    c->P += T;
+    return H2O_OK;
+}
+
+int h2o_step_host(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (T < 1) return fail(c, H2O_ERR_ARG, "T must be >= 1 (got %d)", T);
+    if (!q || !k || !v || !out) return fail(c, H2O_ERR_ARG, "q, k, v, out must be non-NULL");
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t qb = (size_t)c->B * c->Hq * T * c->d * c->elem;
+    const size_t kb = (size_t)c->B * c->Hkv * T * c->d * c->elem;
+    auto up16 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t need = up16(qb) * 2 + up16(kb) * 2;
+    if (need > c->stage_bytes) {
+        H2O_TRY(c, cudaStreamSynchronize(s), "sync before staging growth");
+        cudaFree(c->stage);
+        c->stage = nullptr;
+        c->stage_bytes = 0;
+        H2O_TRY(c, cudaMalloc(&c->stage, need), "cudaMalloc(staging)");
+        c->stage_bytes = need;
+    }
+    char* base = (char*)c->stage;
+    void* dq = base;
+    void* dout = base + up16(qb);
+    void* dk = base + 2 * up16(qb);
+    void* dv = base + 2 * up16(qb) + up16(kb);
+    H2O_TRY(c, cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, s), "copy q to device");
+    H2O_TRY(c, cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, s), "copy k to device");
+    H2O_TRY(c, cudaMemcpyAsync(dv, v, kb, cudaMemcpyHostToDevice, s), "copy v to device");
+    rc = h2o_step(c, dq, dk, dv, dout, T, stream);
+    if (rc != H2O_OK) return rc;
+    H2O_TRY(c, cudaMemcpyAsync(out, dout, qb, cudaMemcpyDeviceToHost, s), "copy out to host");
+    H2O_TRY(c, cudaStreamSynchronize(s), "synchronise after step");
+    return check_ctx(c);
+}
+
+int h2o_scores(h2o_ctx* c, float* dst, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (!dst) return fail(c, H2O_ERR_ARG, "dst is NULL");
+    DeviceGuard g(c->device);
+    H2O_TRY(c, cudaMemcpyAsync(dst, c->scores, sizeof(float) * c->B * c->Hkv * c->C, cudaMemcpyDeviceToDevice,
+                               (cudaStream_t)stream), "copy scores");
+    return H2O_OK;
+}
+
+int h2o_positions(h2o_ctx* c, int32_t* dst, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (!dst) return fail(c, H2O_ERR_ARG, "dst is NULL");
+    DeviceGuard g(c->device);
+    H2O_TRY(c, cudaMemcpyAsync(dst, c->pos, sizeof(int32_t) * c->B * c->Hkv * c->C, cudaMemcpyDeviceToDevice,
+                               (cudaStream_t)stream), "copy positions");
+    return H2O_OK;
+}
+
+int h2o_counters(const h2o_ctx* c, int64_t* P, int64_t* n) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    if (P) *P = c->P;
+    if (n) *n = c->n;
+    return H2O_OK;
+}
+
+int h2o_last_step_info(const h2o_ctx* c, int* T_last, int* n_prev) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    if (T_last) *T_last = c->last_T;
+    if (n_prev) *n_prev = c->last_n;
+    return H2O_OK;
+}
+
+int h2o_candidates(h2o_ctx* c, float* scores, int32_t* pos, uint8_t* kept, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (c->last_T == 0) return fail(c, H2O_ERR_ARG, "no step has run yet");
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t groups = (size_t)c->B * c->Hkv;
+    const size_t nc = (size_t)c->last_n + c->last_T;
+    const size_t src_pitch = (size_t)c->C + c->tmax;
+    if (scores)
+        H2O_TRY(c, cudaMemcpy2DAsync(scores, nc * 4, c->cand_score, src_pitch * 4, nc * 4, groups,
+                                     cudaMemcpyDeviceToDevice, s), "copy candidate scores");
+    if (pos)
+        H2O_TRY(c, cudaMemcpy2DAsync(pos, nc * 4, c->cand_pos, src_pitch * 4, nc * 4, groups,
+                                     cudaMemcpyDeviceToDevice, s), "copy candidate positions");
+    if (kept)
+        H2O_TRY(c, cudaMemcpy2DAsync(kept, nc, c->cand_kept, src_pitch, nc, groups, cudaMemcpyDeviceToDevice, s),
+                "copy kept flags");
+    return H2O_OK;
+}
+
+int h2o_token_slots(h2o_ctx* c, int32_t* dst, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (c->last_T == 0) return fail(c, H2O_ERR_ARG, "no step has run yet");
+    if (!dst) return fail(c, H2O_ERR_ARG, "dst is NULL");
+    DeviceGuard g(c->device);
+    const size_t groups = (size_t)c->B * c->Hkv;
+    H2O_TRY(c, cudaMemcpy2DAsync(dst, (size_t)c->last_T * 4, c->token_slot, (size_t)c->tmax * 4,
+                                 (size_t)c->last_T * 4, groups, cudaMemcpyDeviceToDevice, (cudaStream_t)stream),
+            "copy token slots");
+    return H2O_OK;
+}
+
+int h2o_lse(h2o_ctx* c, float* dst, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (c->last_T == 0) return fail(c, H2O_ERR_ARG, "no step has run yet");
+    if (!dst) return fail(c, H2O_ERR_ARG, "dst is NULL");
+    DeviceGuard g(c->device);
+    const size_t rows = (size_t)c->B * c->Hq;
+    H2O_TRY(c, cudaMemcpy2DAsync(dst, (size_t)c->last_T * 4, c->lse, (size_t)c->tmax * 4, (size_t)c->last_T * 4,
+                                 rows, cudaMemcpyDeviceToDevice, (cudaStream_t)stream), "copy lse");
+    return H2O_OK;
+}
+
+int h2o_get_state(h2o_ctx* c, void* K, void* V, float* scores, int32_t* positions, int64_t* P, int64_t* n,
+                  void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t groups = (size_t)c->B * c->Hkv;
+    const size_t cb = groups * c->C * c->d * c->elem;
+    if (K) H2O_TRY(c, cudaMemcpyAsync(K, c->Kc, cb, cudaMemcpyDeviceToDevice, s), "copy K");
+    if (V) H2O_TRY(c, cudaMemcpyAsync(V, c->Vc, cb, cudaMemcpyDeviceToDevice, s), "copy V");
+    if (scores) H2O_TRY(c, cudaMemcpyAsync(scores, c->scores, groups * c->C * 4, cudaMemcpyDeviceToDevice, s), "copy scores");
+    if (positions) H2O_TRY(c, cudaMemcpyAsync(positions, c->pos, groups * c->C * 4, cudaMemcpyDeviceToDevice, s), "copy positions");
+    if (P) *P = c->P;
+    if (n) *n = c->n;
+    return H2O_OK;
+}
+
+int h2o_set_state(h2o_ctx* c, const void* K, const void* V, const float* scores, const int32_t* positions,
+                  int64_t P, int64_t n, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (!K || !V || !scores || !positions) return fail(c, H2O_ERR_ARG, "K, V, scores, positions must be non-NULL");
+    if (P < 0 || P > (int64_t)INT32_MAX || n < 0 || n > c->C || n > P)
+        return fail(c, H2O_ERR_ARG, "need 0 <= n <= min(C, P) and P < 2^31");
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t groups = (size_t)c->B * c->Hkv;
+    std::vector<int32_t> hp(groups * c->C);
+    H2O_TRY(c, cudaMemcpyAsync(hp.data(), positions, hp.size() * 4, cudaMemcpyDeviceToHost, s), "read positions");
+    H2O_TRY(c, cudaStreamSynchronize(s), "sync set_state");
+    std::vector<int32_t> sorted((size_t)n);
+    for (size_t gi = 0; gi < groups; ++gi) {
+        const int32_t* p = hp.data() + gi * c->C;
+        for (int64_t j = 0; j < n; ++j) {
+            if (p[j] < 0 || p[j] >= P)
+                return fail(c, H2O_ERR_ARG, "group %zu slot %lld: position %d outside [0, P)", gi, (long long)j, p[j]);
+            sorted[j] = p[j];
+        }
+        for (int64_t j = n; j < c->C; ++j)
+            if (p[j] != -1) return fail(c, H2O_ERR_ARG, "group %zu slot %lld beyond n must be empty (-1)", gi, (long long)j);
+        std::sort(sorted.begin(), sorted.end());
+        if (std::adjacent_find(sorted.begin(), sorted.end()) != sorted.end())
+            return fail(c, H2O_ERR_ARG, "group %zu has duplicate positions", gi);
+    }
+    const size_t cb = groups * c->C * c->d * c->elem;
+    H2O_TRY(c, cudaMemcpyAsync(c->Kc, K, cb, cudaMemcpyDeviceToDevice, s), "copy K");
+    H2O_TRY(c, cudaMemcpyAsync(c->Vc, V, cb, cudaMemcpyDeviceToDevice, s), "copy V");
+    H2O_TRY(c, cudaMemcpyAsync(c->scores, scores, groups * c->C * 4, cudaMemcpyDeviceToDevice, s), "copy scores");
+    H2O_TRY(c, cudaMemcpyAsync(c->pos, positions, groups * c->C * 4, cudaMemcpyDeviceToDevice, s), "copy positions");
+    c->P = P;
+    c->n = n;
+    c->last_T = 0;
+    return H2O_OK;
+}
+
+int h2o_sync_check(h2o_ctx* c, void* stream) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    DeviceGuard g(c->device);
+    H2O_TRY(c, cudaStreamSynchronize((cudaStream_t)stream), "synchronise");
+    return check_ctx(c);
+}
+
+int h2o_profile_begin(h2o_ctx* c, int max_steps) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (max_steps < 1) return fail(c, H2O_ERR_ARG, "max_steps must be >= 1");
+    DeviceGuard g(c->device);
+    for (cudaEvent_t e : c->prof_ev) cudaEventDestroy(e);
+    c->prof_ev.assign((size_t)max_steps * (kMaxStepKernels + 1), nullptr);
+    for (auto& e : c->prof_ev) H2O_TRY(c, cudaEventCreate(&e), "cudaEventCreate");
+    c->prof_logs.assign(max_steps, LaunchLog());
+    c->prof_max_steps = max_steps;
+    c->prof_steps = 0;
+    c->prof_on = true;
+    return H2O_OK;
+}
+
+int h2o_profile_end(h2o_ctx* c, int max_kernels, const char** names, double* total_ms, int* launches) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    if (!c->prof_on) return fail(c, H2O_ERR_ARG, "profiling was not started");
+    DeviceGuard g(c->device);
+    c->prof_on = false;
+    int nk = 0;
+    std::vector<const char*> nm;
+    std::vector<double> ms;
+    std::vector<int> cnt;
+    for (int st = 0; st < c->prof_steps; ++st) {
+        const LaunchLog& L = c->prof_logs[st];
+        for (int i = 0; i < L.n; ++i) {
+            cudaEvent_t a = c->prof_ev[(size_t)st * (kMaxStepKernels + 1) + i];
+            cudaEvent_t b = c->prof_ev[(size_t)st * (kMaxStepKernels + 1) + i + 1];
+            H2O_TRY(c, cudaEventSynchronize(b), "cudaEventSynchronize");
+            float t = 0.f;
+            H2O_TRY(c, cudaEventElapsedTime(&t, a, b), "cudaEventElapsedTime");
+            int idx = -1;
+            for (int j = 0; j < (int)nm.size(); ++j)
+                if (strcmp(nm[j], L.names[i]) == 0) idx = j;
+            if (idx < 0) {
+                nm.push_back(L.names[i]);
+                ms.push_back(0.0);
+                cnt.push_back(0);
+                idx = (int)nm.size() - 1;
+            }
+            ms[idx] += t;
+            cnt[idx] += 1;
+        }
+    }
+    for (cudaEvent_t e : c->prof_ev) cudaEventDestroy(e);
+    c->prof_ev.clear();
+    c->prof_logs.clear();
+    nk = (int)nm.size();
+    for (int j = 0; j < nk && j < max_kernels; ++j) {
+        if (names) names[j] = nm[j];
+        if (total_ms) total_ms[j] = ms[j];
+        if (launches) launches[j] = cnt[j];
+    }
+    return nk;
+}
+
+int h2o_selftest_wait(h2o_ctx* c, int spins, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    DeviceGuard g(c->device);
+    WaitBound wb;
+    wb.err_word = c->err_dev;
+    wb.ns = (unsigned long long)(spins > 0 ? spins : 1) * 1000000ull;  // spins read as milliseconds
+    H2O_TRY(c, launch_wait_selftest(wb, (cudaStream_t)stream), "launch wait self-test");
+    H2O_TRY(c, cudaStreamSynchronize((cudaStream_t)stream), "synchronise wait self-test");
+    return check_ctx(c);
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// kernels.h -- internal launch interface of the H2O step kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace h2o {
+
+// Names (and, when profiling, events) of the kernels one step launches.
+// Every launcher calls done() right after each of its launches.
+constexpr int kMaxStepKernels = 8;
+struct LaunchLog {
+    cudaEvent_t* ev = nullptr;   // kMaxStepKernels + 1 events, or nullptr
+    const char* names[kMaxStepKernels];
+    int n = 0;
+    void done(const char* name, cudaStream_t s) {
+        if (n >= kMaxStepKernels) return;
+        names[n++] = name;
+        if (ev) cudaEventRecord(ev[n], s);
+    }
+};
+
+// Everything one step's kernels read or write. Device pointers unless noted.
+struct StepArgs {
+    int B, Hq, Hkv, d, C, T;
+    int n;            // valid cache slots (prefix 0..n-1) before the step
+    int64_t P;        // position of the chunk's first token
+    int dtype;        // 0 = bf16, 1 = fp32
+    int tmax;         // capacity (in tokens) of the per-step workspace
+    const void* q;    // [B,Hq,T,d]
+    const void* k;    // [B,Hkv,T,d]
+    const void* v;    // [B,Hkv,T,d]
+    void* out;        // [B,Hq,T,d]
+    void* Kc;         // [B,Hkv,C,d] cache keys
+    void* Vc;         // [B,Hkv,C,d] cache values
+    float* scores;    // [B,Hkv,C]
+    int32_t* pos;     // [B,Hkv,C]
+    float* lse;       // [B,Hq,tmax] natural-log normaliser per row
+    float* cand_score;   // [B,Hkv,C+tmax]
+    int32_t* cand_pos;   // [B,Hkv,C+tmax]
+    uint8_t* cand_kept;  // [B,Hkv,C+tmax]
+    int32_t* token_slot; // [B,Hkv,tmax]
+    int32_t* free_list;  // [B,Hkv,C]
+    float* partials;     // weight-sum partials (tensor-core path)
+    size_t partial_elems;
+    const void* tmaps;   // device copy of the step's TMA descriptors (tensor-core path)
+    WaitBound wb;
+    cudaStream_t stream;
+    int num_sms;
+    LaunchLog* log;
+};
+
+inline int cand_stride(const StepArgs& a) { return a.C + a.tmax; }
+
+// SIMT kernels (fp32 path; any supported d).
+cudaError_t launch_sdpa_simt(const StepArgs& a);
+cudaError_t launch_wsum_simt(const StepArgs& a);
+// Eviction: per (sequence, KV head) radix select + slot map, then K/V copy.
+cudaError_t launch_select(const StepArgs& a);
+cudaError_t launch_scatter(const StepArgs& a);
+// Self-test of the bounded wait.
+cudaError_t launch_wait_selftest(const WaitBound& wb, cudaStream_t s);
+
+}  // namespace h2o

@@ -1,0 +1,19 @@
+// tc.h -- tensor-core (tcgen05 / TMEM / TMA) kernels of the bf16 H2O step.
+#pragma once
+
+#include "kernels.h"
+
+namespace h2o {
+
+// True when the device is sm_100 and the head dimension has a tensor-core path.
+bool tc_supported(int device, int d);
+// Workspace floats the weight-sum partials need for chunks of up to tmax tokens.
+size_t tc_partial_elems(int B, int Hq, int Hkv, int C, int tmax);
+// Names of the tensor-core kernels one step launches (returns the count).
+int tc_kernel_plan(int B, int Hq, int Hkv, int d, int C, int T, int n, const char** names, int max_names);
+// Chunk SDPA: O and per-row LSE.
+cudaError_t tc_sdpa(const StepArgs& a);
+// Per-key weight sums added to the scores (writes cand_score / cand_pos).
+cudaError_t tc_wsum(const StepArgs& a);
+
+}  // namespace h2o

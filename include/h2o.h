@@ -1,0 +1,192 @@
+/*
+ * h2o.h -- C ABI of the B200 (sm_100a) chunked H2O sparse-attention step.
+ *
+ * The operation is the heavy-hitter (H2O) KV-cache step of "Learning how to
+ * Forget: Fine-tuning for Long-Context Sparse Attention" (arXiv 2608.19920):
+ *   - paper page, section "Kernel Support Needs": attention kernels should
+ *     return, beside the SDPA output, the summed attention weights
+ *     sum_i w[b,h,i,j] of every key slot j, under the positional mask
+ *     (b,h,i,j) -> -inf * I[P + i < t(b,h,j)];
+ *   - paper page, section "Improvements to Heavy-Hitter Oracle (H2O)": a
+ *     slot's H2O score accumulates those sums, and new content overwrites the
+ *     slots with the smallest scores.
+ * One call of h2o_step processes one chunk of T new tokens per sequence:
+ *   1. SDPA of the chunk's queries against the C-slot cache plus the chunk
+ *      itself (cache fully visible, causal inside the chunk, diagonal
+ *      included), softmax scale 1/sqrt(d), GQA: query head h reads KV head
+ *      h / (Hq / Hkv);
+ *   2. per KV head, the weight every candidate key received, summed over the
+ *      chunk's rows and over the Hq/Hkv query heads of the group, is added to
+ *      its score (cache slots: old score + sum; chunk tokens: the sum);
+ *   3. per (sequence, KV head), of the n valid slots plus T chunk tokens the C
+ *      with the largest score survive (equal scores: the larger position
+ *      survives); kept cache entries stay in their slots, and the kept chunk
+ *      tokens, in position order, fill the free slots in ascending slot order.
+ *
+ * Conventions for every entry point:
+ *   - Every call returns a status (H2O_OK or a negative H2O_ERR_*); none
+ *     aborts the process. h2o_last_error() describes the last failure.
+ *   - Pointers named "device" are CUDA device pointers of the context's
+ *     device; "host" pointers are host memory. The caller owns every buffer it
+ *     passes; the library owns the cache and its workspace.
+ *   - "stream" is a cudaStream_t (NULL = the legacy default stream). Calls are
+ *     asynchronous and stream-ordered unless stated otherwise; buffers passed
+ *     to a call must stay valid until the stream reaches it.
+ *   - Layouts are dense row-major (C order), element type H2O_BF16
+ *     (bfloat16) or H2O_FP32 (float) as chosen at creation:
+ *       q, out [B, Hq,  T, d]      k, v [B, Hkv, T, d]
+ *       cache  [B, Hkv, C, d]      scores (float) / positions (int32) [B, Hkv, C]
+ *     q, k, v, out must be 16-byte aligned.
+ *   - Supported shapes: d in {64, 128}; Hq % Hkv == 0; C >= 1; T >= 1;
+ *     positions stay below 2^31. All sequences of the batch advance together:
+ *     the chunk of a call holds positions P .. P+T-1 of every sequence.
+ *   - The valid cache slots of every (sequence, KV head) are always the
+ *     prefix 0 .. n-1, with n = min(C, tokens processed); every state the
+ *     library produces has this form and h2o_set_state() rejects others.
+ *   - A kernel that waits longer than its bound (H2O_WAIT_TIMEOUT_MS below)
+ *     stops, records the fact in a device-visible error word and returns;
+ *     the next call on that context reports H2O_ERR_TIMEOUT and the context
+ *     is poisoned (every later call returns H2O_ERR_POISONED).
+ */
+#ifndef H2O_H_
+#define H2O_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct h2o_ctx h2o_ctx;
+
+enum h2o_status {
+    H2O_OK = 0,
+    H2O_ERR_ARG = -1,         /* bad argument, shape or state */
+    H2O_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+    H2O_ERR_OOM = -3,         /* device or host allocation failed */
+    H2O_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed */
+    H2O_ERR_TIMEOUT = -5,     /* a device-side wait ran out of its bound */
+    H2O_ERR_POISONED = -6,    /* an earlier device error: context unusable */
+    H2O_ERR_UNSUPPORTED = -7  /* shape outside the supported set */
+};
+
+enum h2o_dtype { H2O_BF16 = 0, H2O_FP32 = 1 };
+
+/* Create a bf16 context on the current CUDA device: an empty cache of C slots
+ * per (sequence, KV head), P = 0. Allocates all device memory it will need for
+ * chunks of up to T = C tokens (larger chunks grow the workspace once).
+ * *out receives the handle, NULL on failure. */
+int h2o_create(int B, int Hq, int Hkv, int d, int C, h2o_ctx **out);
+
+/* As h2o_create, with the element type (enum h2o_dtype) and the largest
+ * chunk length to size the workspace for (max_T >= 1). */
+int h2o_create_ex(int B, int Hq, int Hkv, int d, int C, int dtype, int max_T, h2o_ctx **out);
+
+/* Free every resource of the context (synchronises its device first).
+ * NULL is accepted. */
+int h2o_destroy(h2o_ctx *ctx);
+
+/* One H2O step on the chunk (q, k, v) of T tokens (device pointers, layouts
+ * above); writes the attention output to out (device). Updates the cache,
+ * scores and positions; P advances by T. Asynchronous on `stream`. */
+int h2o_step(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
+             int T, void *stream);
+
+/* h2o_step with HOST buffers: copies q, k, v to library-owned device staging
+ * buffers, runs the step and copies the output back into out (host). Page-
+ * locked host memory gives asynchronous copies; pageable memory works too.
+ * Returns after the output has arrived in out (synchronises `stream`). */
+int h2o_step_host(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
+                  int T, void *stream);
+
+/* Current H2O scores, float [B, Hkv, C] (device dst); 0 in empty slots. */
+int h2o_scores(h2o_ctx *ctx, float *dst, void *stream);
+
+/* Current slot positions, int32 [B, Hkv, C] (device dst); -1 = empty. */
+int h2o_positions(h2o_ctx *ctx, int32_t *dst, void *stream);
+
+/* Host-side counters: *P = tokens processed per sequence, *n = valid slots
+ * per (sequence, KV head). Either pointer may be NULL. No synchronisation. */
+int h2o_counters(const h2o_ctx *ctx, int64_t *P, int64_t *n);
+
+/* Description of the last failure on this context (ctx = NULL: the last
+ * failure of this thread that had no context, e.g. in h2o_create). */
+const char *h2o_last_error(const h2o_ctx *ctx);
+
+/* ---- inspection, checkpoint and test hooks ---------------------------- */
+
+/* Candidates of the last step, for each (sequence, KV head): index c < n_prev
+ * is cache slot c, index n_prev + t is chunk token t, with n_prev the valid
+ * slot count before that step. scores: updated score (old + weight sum);
+ * pos: position; kept: 1 if it survived. Device arrays of [B, Hkv, ncand]
+ * with ncand = n_prev + T_last (query it with h2o_last_step_info). Any of the
+ * three pointers may be NULL. */
+int h2o_candidates(h2o_ctx *ctx, float *scores, int32_t *pos, uint8_t *kept, void *stream);
+
+/* Slot each chunk token of the last step was written to, -1 if dropped:
+ * device int32 [B, Hkv, T_last]. */
+int h2o_token_slots(h2o_ctx *ctx, int32_t *dst, void *stream);
+
+/* Natural-log softmax normaliser (log-sum-exp of the scaled logits) of every
+ * query row of the last step: device float [B, Hq, T_last]. */
+int h2o_lse(h2o_ctx *ctx, float *dst, void *stream);
+
+/* T and the pre-step valid count n_prev of the last step (host ints). */
+int h2o_last_step_info(const h2o_ctx *ctx, int *T_last, int *n_prev);
+
+/* Export the cache: K, V [B, Hkv, C, d] (context dtype), scores float and
+ * positions int32 [B, Hkv, C] (device pointers, any may be NULL), and the
+ * counters P and n (host int64, may be NULL). */
+int h2o_get_state(h2o_ctx *ctx, void *K, void *V, float *scores, int32_t *positions,
+                  int64_t *P, int64_t *n, void *stream);
+
+/* Import a cache exported by h2o_get_state (or built by the caller). Checks,
+ * on the host after copying positions back (synchronises `stream`): for every
+ * (sequence, KV head) positions[0..n-1] are distinct values in [0, P) and
+ * positions[n..C-1] are -1; 0 <= n <= min(C, P). On success the next step
+ * processes positions P .. P+T-1. Device pointers; P, n by value. */
+int h2o_set_state(h2o_ctx *ctx, const void *K, const void *V, const float *scores,
+                  const int32_t *positions, int64_t P, int64_t n, void *stream);
+
+/* Empty the cache and set P = 0 (asynchronous on `stream`). */
+int h2o_reset(h2o_ctx *ctx, void *stream);
+
+/* Check the context's device error word after synchronising `stream`;
+ * returns H2O_OK, or H2O_ERR_TIMEOUT (and poisons the context). */
+int h2o_sync_check(h2o_ctx *ctx, void *stream);
+
+/* Self-test of the bounded device wait: launches one block that waits on a
+ * shared-memory barrier nothing will complete, giving up after timeout_ms
+ * milliseconds, synchronises `stream` and returns what the context's error
+ * word reports (H2O_ERR_TIMEOUT when the bound works). No memory traffic is
+ * in flight during the wait. Poisons the context, as any timeout does. */
+int h2o_selftest_wait(h2o_ctx *ctx, int timeout_ms, void *stream);
+
+/* Per-kernel timing (tracing). h2o_profile_begin allocates CUDA events for
+ * up to max_steps steps and makes every following h2o_step record an event
+ * on its stream before its first kernel and after each kernel. h2o_profile_end
+ * synchronises those events, stops recording and reports, per kernel name
+ * (in launch order of a step), the summed device time in milliseconds and the
+ * number of launches. names/total_ms/launches are host arrays of max_kernels
+ * entries; returns the number of kernel names (>= 0) or an error. */
+int h2o_profile_begin(h2o_ctx *ctx, int max_steps);
+int h2o_profile_end(h2o_ctx *ctx, int max_kernels, const char **names, double *total_ms,
+                    int *launches);
+
+/* Library build identifier (static string). */
+const char *h2o_version(void);
+
+/* Per-step kernel launches issued by h2o_step for this context (host int);
+ * fills names (static strings) up to max_names. */
+int h2o_kernel_plan(const h2o_ctx *ctx, int T, const char **names, int max_names);
+
+#ifdef __cplusplus
+}
+#endif
+
+/* Environment knobs (read at h2o_create):
+ *   H2O_WAIT_TIMEOUT_MS  how long a kernel polls an mbarrier before it gives
+ *                        up (default 2000 ms); values < 1 are ignored.
+ */
+#endif /* H2O_H_ */
