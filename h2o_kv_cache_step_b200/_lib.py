@@ -53,6 +53,7 @@ SIGNATURES = [
     ("h2o_selftest_wait", _I, [_P, _I, _P]),
     ("h2o_version", ctypes.c_char_p, []),
     ("h2o_kernel_plan", _I, [_P, _I, ctypes.POINTER(ctypes.c_char_p), _I]),
+    ("h2o_select_noalloc", _I, [_I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, _P]),
     ("h2o_profile_begin", _I, [_P, _I]),
     ("h2o_profile_end", _I, [_P, _I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
                              ctypes.POINTER(_I)]),

@@ -39,6 +39,10 @@ void set_thread_err(const char* fmt, ...) {
 
 }  // namespace
 
+void h2o::set_thread_error_message(const char* msg) {
+    snprintf(g_thread_err, sizeof(g_thread_err), "%s", msg);
+}
+
 struct h2o_ctx {
     int B, Hq, Hkv, d, C, dtype, tmax;
     int device;

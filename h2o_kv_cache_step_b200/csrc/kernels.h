@@ -60,6 +60,8 @@ cudaError_t launch_wsum_simt(const StepArgs& a);
 // Eviction: per (sequence, KV head) radix select + slot map, then K/V copy.
 cudaError_t launch_select(const StepArgs& a);
 cudaError_t launch_scatter(const StepArgs& a);
+// Sets the message h2o_last_error(NULL) reports on this thread.
+void set_thread_error_message(const char* msg);
 // Self-test of the bounded wait.
 cudaError_t launch_wait_selftest(const WaitBound& wb, cudaStream_t s);
 

@@ -174,6 +174,32 @@ int h2o_profile_begin(h2o_ctx *ctx, int max_steps);
 int h2o_profile_end(h2o_ctx *ctx, int max_kernels, const char **names, double *total_ms,
                     int *launches);
 
+/* Eviction alone, without any device allocation. The paper has no
+ * counterpart of this entry point; it exists for callers that cannot call
+ * cudaMalloc -- plugin hosts and serving runtimes that only hand out buffers
+ * they pre-allocated under a fixed memory budget, and latency-critical paths
+ * where an allocation would synchronise the device.
+ * Given, for `groups` (sequence, KV head) groups, the updated candidate scores
+ * and positions of one step (device float / int32 [groups, n+T]: cache slots
+ * 0..n-1, then the T chunk tokens at positions P..P+T-1), it computes what
+ * h2o_step's eviction computes: kept flags (device uint8 [groups, n+T]), the
+ * slot of each chunk token or -1 (device int32 [groups, T]), and updates the
+ * slot scores and positions (device float / int32 [groups, C], in/out: kept
+ * cache slots take their new score, kept chunk tokens fill the free slots in
+ * ascending order, leftover free slots become empty). The caller owns every
+ * buffer. Scratch (the free-slot lists) lives in a static device array of
+ * 262144 int32 (1 MiB) that every GPU loading the library holds until exit;
+ * groups * C above that returns H2O_ERR_UNSUPPORTED. The first call on a
+ * device looks up that array's device address (once per device); make that
+ * first call before any stream capture. Each device has its own copy of the
+ * array and every call on that device shares it, keeping whatever the last
+ * call left there: calls that overlap on the GPU (for example on two streams)
+ * race, so serialise them. Nothing in it needs clearing between calls. Asynchronous on `stream`; errors are
+ * described by h2o_last_error(NULL). */
+int h2o_select_noalloc(int groups, int C, int n, int T, int64_t P, const float *cand_score,
+                       const int32_t *cand_pos, float *scores, int32_t *positions, uint8_t *kept,
+                       int32_t *token_slot, void *stream);
+
 /* Library build identifier (static string). */
 const char *h2o_version(void);
 
