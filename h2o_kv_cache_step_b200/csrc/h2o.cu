@@ -30,13 +30,6 @@ namespace {
 
 thread_local char g_thread_err[512] = "";
 
-void set_thread_err(const char* fmt, ...) {
-    va_list ap;
-    va_start(ap, fmt);
-    vsnprintf(g_thread_err, sizeof(g_thread_err), fmt, ap);
-    va_end(ap);
-}
-
 }  // namespace
 
 void h2o::set_thread_error_message(const char* msg) {
@@ -350,6 +343,7 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
         a.log->ev = &c->prof_ev[(size_t)slot * (kMaxStepKernels + 1)];
         H2O_TRY(c, cudaEventRecord(a.log->ev[0], s), "record profiling event");
     }
+    a.nparts = c->use_tc ? tc_partial_count(c->Hq, c->Hkv, T) : 0;
     if (c->use_tc) {
         H2O_TRY(c, tc_sdpa(a), "launch tensor-core SDPA");
         H2O_TRY(c, tc_wsum(a), "launch tensor-core weight sums");

@@ -43,8 +43,9 @@ struct StepArgs {
     uint8_t* cand_kept;  // [B,Hkv,C+tmax]
     int32_t* token_slot; // [B,Hkv,tmax]
     int32_t* free_list;  // [B,Hkv,C]
-    float* partials;     // weight-sum partials (tensor-core path)
+    float* partials;     // weight-sum partials [nparts][B*Hkv][C+tmax] (tensor-core path)
     size_t partial_elems;
+    int nparts;          // > 0: the selection kernel first sums the partials
     const void* tmaps;   // device copy of the step's TMA descriptors (tensor-core path)
     WaitBound wb;
     cudaStream_t stream;

@@ -65,10 +65,10 @@ __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
 }
 
 __global__ void __launch_bounds__(kSelThreads)
-select_kernel(const float* __restrict__ cand_score, const int32_t* __restrict__ cand_pos,
+select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
               uint8_t* __restrict__ cand_kept, int32_t* __restrict__ token_slot,
               int32_t* __restrict__ free_list, float* __restrict__ scores, int32_t* __restrict__ pos,
-              int C, int T, int n, int tmax, long long P) {
+              const float* __restrict__ partials, int nparts, int C, int T, int n, int tmax, long long P) {
     __shared__ unsigned int hist[256];
     __shared__ int scan_scratch[33];
     __shared__ unsigned long long sh_prefix;
@@ -76,13 +76,25 @@ select_kernel(const float* __restrict__ cand_score, const int32_t* __restrict__ 
 
     const size_t bg = blockIdx.x;
     const int m = n + T;
-    const float* cs = cand_score + bg * (size_t)(C + tmax);
-    const int32_t* cp = cand_pos + bg * (size_t)(C + tmax);
+    float* cs = cand_score + bg * (size_t)(C + tmax);
+    int32_t* cp = cand_pos + bg * (size_t)(C + tmax);
     uint8_t* kept = cand_kept + bg * (size_t)(C + tmax);
     int32_t* fl = free_list + bg * (size_t)C;
     int32_t* ts = token_slot + bg * (size_t)tmax;
     float* sc = scores + bg * (size_t)C;
     int32_t* ps = pos + bg * (size_t)C;
+
+    // ---- 0. candidate scores from the weight-sum partials (fixed part order)
+    if (nparts > 0) {
+        const size_t pstride = (size_t)gridDim.x * (C + tmax);
+        for (int c = threadIdx.x; c < m; c += blockDim.x) {
+            float s = c < n ? sc[c] : 0.f;
+            for (int q = 0; q < nparts; ++q) s += partials[q * pstride + bg * (size_t)(C + tmax) + c];
+            cs[c] = s;
+            cp[c] = c < n ? ps[c] : (int32_t)(P + (c - n));
+        }
+        __syncthreads();
+    }
 
     // ---- 1. threshold: the C-th largest key (radix select, 8 bits a pass)
     if (threadIdx.x == 0) {
@@ -226,8 +238,8 @@ __global__ void wait_selftest_kernel(WaitBound wb) {
 
 cudaError_t launch_select(const StepArgs& a) {
     select_kernel<<<a.B * a.Hkv, kSelThreads, 0, a.stream>>>(
-        a.cand_score, a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, a.C, a.T, a.n,
-        a.tmax, (long long)a.P);
+        a.cand_score, a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, a.partials, a.nparts,
+        a.C, a.T, a.n, a.tmax, (long long)a.P);
     a.log->done("select_kernel", a.stream);
     return cudaGetLastError();
 }

@@ -9,6 +9,8 @@ namespace h2o {
 bool tc_supported(int device, int d);
 // Workspace floats the weight-sum partials need for chunks of up to tmax tokens.
 size_t tc_partial_elems(int B, int Hq, int Hkv, int C, int tmax);
+// Number of weight-sum partials (row parts) a chunk of T tokens produces.
+int tc_partial_count(int Hq, int Hkv, int T);
 // Names of the tensor-core kernels one step launches (returns the count).
 int tc_kernel_plan(int B, int Hq, int Hkv, int d, int C, int T, int n, const char** names, int max_names);
 // Chunk SDPA: O and per-row LSE.
