@@ -169,6 +169,19 @@ def run_ours(args, rank, world, local_rank):
         for (q, k, v) in chunks:
             cache.step(q, k, v, out=out)
 
+    if args.mode == "chunk":
+        # one steady-state chunk step per bench step (for profiler captures):
+        # a full cache, then chunk C/T+1 of the sequence
+        K0, V0, S0, pos0 = synth.random_state(wl, n=wl.C, P=(wl.C // wl.T + 1) * wl.T, seed=1)
+        st = tuple(torch.from_numpy(x).to(dev) for x in (K0, V0, S0, pos0))
+        st = (st[0].to(tdt), st[1].to(tdt), st[2], st[3])
+        c_idx = min(wl.n_chunks - 1, wl.C // wl.T + 1)
+        sched = [(wl.C, wl.T)]
+
+        def prefill():  # noqa: F811
+            cache.set_state(*st, P=c_idx * wl.T, n=wl.C)
+            cache.step(*chunks[c_idx], out=out)
+
     for _ in range(args.warmup):
         prefill()
     cache.sync_check()
@@ -180,7 +193,7 @@ def run_ours(args, rank, world, local_rank):
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    cache.profile_begin(args.steps * wl.n_chunks)
+    cache.profile_begin(args.steps * len(sched))
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -203,7 +216,7 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_total = float(t.item())
     ms_per_step = ms_total / args.steps
-    tokens = wl.B * wl.N * args.steps * world
+    tokens = (wl.B * wl.N if args.mode == "prefill" else wl.B * wl.T) * args.steps * world
     value = tokens / (ms_total / 1e3)
 
     # roofline of the dominant kernel
@@ -254,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through h2o_step_host with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.mode == "prefill":
         host = [tuple(t.cpu().pin_memory() for t in ch) for ch in chunks]
         hout = torch.empty_like(chunks[0][0], device="cpu").pin_memory()
         h2d = sum(t.numel() * t.element_size() for ch in host for t in ch)
@@ -398,6 +411,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "chunk"],
+                    help="prefill: a bench step is a whole-sequence prefill (default); chunk: one "
+                         "steady-state chunk step (for profiler captures)")
     ap.add_argument("--cpu-groups", type=int, default=0,
                     help="KV groups in the oracle sample (default: host cores)")
     args = ap.parse_args()

@@ -51,6 +51,7 @@ SIGNATURES = [
     ("h2o_reset", _I, [_P, _P]),
     ("h2o_sync_check", _I, [_P, _P]),
     ("h2o_selftest_wait", _I, [_P, _I, _P]),
+    ("h2o_selftest_exp2", _I, [_P, _P, _P, _P, _I, _P]),
     ("h2o_version", ctypes.c_char_p, []),
     ("h2o_kernel_plan", _I, [_P, _I, ctypes.POINTER(ctypes.c_char_p), _I]),
     ("h2o_select_noalloc", _I, [_I, _I, _I, _I, _I64, _P, _P, _P, _P, _P, _P, _P]),

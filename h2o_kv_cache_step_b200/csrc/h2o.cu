@@ -593,6 +593,15 @@ int h2o_profile_end(h2o_ctx* c, int max_kernels, const char** names, double* tot
     return nk;
 }
 
+int h2o_selftest_exp2(const float* x, float* y_poly3, float* y_poly4, float* y_mufu, int n, void* stream) {
+    if (n < 0 || (n > 0 && (!x || !y_poly3 || !y_poly4 || !y_mufu)))
+        return fail(nullptr, H2O_ERR_ARG, "h2o_selftest_exp2: bad arguments");
+    if (n == 0) return H2O_OK;
+    H2O_TRY(nullptr, tc_exp2_selftest(x, y_poly3, y_poly4, y_mufu, n, (cudaStream_t)stream),
+            "launch exp2 self-test");
+    return H2O_OK;
+}
+
 int h2o_selftest_wait(h2o_ctx* c, int spins, void* stream) {
     int rc = check_ctx(c);
     if (rc != H2O_OK) return rc;

@@ -34,6 +34,10 @@ __device__ __forceinline__ uint64_t cand_key(const float* cs, const int32_t* cp,
     return ((uint64_t)ordered_bits(cs[c]) << 32) | (uint32_t)cp[c];
 }
 
+// Candidate keys are staged in shared memory when they fit (the radix passes
+// then read them from there), otherwise rebuilt from global memory per pass.
+constexpr int kSmemKeyLimit = 24576;  // 192 KB of 64-bit keys
+
 // Exclusive prefix sum of one int per thread over the block; *total gets the
 // sum. Uses `scratch` (>= 33 ints of shared memory).
 __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
@@ -64,6 +68,7 @@ __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
     return r;
 }
 
+template <bool SMEM_KEYS>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
               uint8_t* __restrict__ cand_kept, int32_t* __restrict__ token_slot,
@@ -73,6 +78,7 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     __shared__ int scan_scratch[33];
     __shared__ unsigned long long sh_prefix;
     __shared__ int sh_shift, sh_krem, sh_done;
+    extern __shared__ unsigned long long skeys[];  // [m] when SMEM_KEYS
 
     const size_t bg = blockIdx.x;
     const int m = n + T;
@@ -95,6 +101,11 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         }
         __syncthreads();
     }
+    if (SMEM_KEYS) {
+        for (int c = threadIdx.x; c < m; c += blockDim.x) skeys[c] = cand_key(cs, cp, c);
+        __syncthreads();
+    }
+    auto key_of = [&](int c) -> uint64_t { return SMEM_KEYS ? (uint64_t)skeys[c] : cand_key(cs, cp, c); };
 
     // ---- 1. threshold: the C-th largest key (radix select, 8 bits a pass)
     if (threadIdx.x == 0) {
@@ -110,7 +121,7 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0u;
         __syncthreads();
         for (int c = threadIdx.x; c < m; c += blockDim.x) {
-            const uint64_t key = cand_key(cs, cp, c);
+            const uint64_t key = key_of(c);
             const bool match = (shift == 56) || ((key >> (shift + 8)) == prefix);
             if (match) atomicAdd(&hist[(key >> shift) & 255u], 1u);
         }
@@ -157,7 +168,7 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     for (int c = threadIdx.x; c < m; c += blockDim.x) {
         bool k = keep_all;
         if (!keep_all) {
-            const uint64_t key = cand_key(cs, cp, c);
+            const uint64_t key = key_of(c);
             k = fshift >= 64 ? true : ((key >> fshift) >= fprefix);
         }
         kept[c] = (uint8_t)k;
@@ -237,9 +248,23 @@ __global__ void wait_selftest_kernel(WaitBound wb) {
 }  // namespace
 
 cudaError_t launch_select(const StepArgs& a) {
-    select_kernel<<<a.B * a.Hkv, kSelThreads, 0, a.stream>>>(
-        a.cand_score, a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, a.partials, a.nparts,
-        a.C, a.T, a.n, a.tmax, (long long)a.P);
+    const int m = a.n + a.T;
+    if (m <= kSmemKeyLimit) {
+        static int configured = 0;
+        if (!configured) {
+            cudaError_t e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kSmemKeyLimit * 8);
+            if (e != cudaSuccess) return e;
+            configured = 1;
+        }
+        select_kernel<true><<<a.B * a.Hkv, kSelThreads, (size_t)m * 8, a.stream>>>(
+            a.cand_score, a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, a.partials,
+            a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
+    } else {
+        select_kernel<false><<<a.B * a.Hkv, kSelThreads, 0, a.stream>>>(
+            a.cand_score, a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, a.partials,
+            a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
+    }
     a.log->done("select_kernel", a.stream);
     return cudaGetLastError();
 }

@@ -45,6 +45,16 @@ using tc::fence_before_sync;
 constexpr int kThreads = 192;
 constexpr int kRowsPerPart = 1024;   // weight-sum rows per CTA (8 tiles of 128)
 constexpr float kRescaleThreshold = 8.f;  // log2 units
+// Of every 8 columns, how many take the FMA-pipe exp2 instead of the MUFU
+// unit (the MUFU is the other bottleneck next to the tensor core).
+#ifndef H2O_POLY_SDPA
+#define H2O_POLY_SDPA 1
+#endif
+#ifndef H2O_POLY_WSUM
+#define H2O_POLY_WSUM 2
+#endif
+constexpr int kPolyPairsOf4Sdpa = H2O_POLY_SDPA;  // SDPA: pairs in every 4 on the FMA pipe
+constexpr int kPolyPairsOf8Wsum = H2O_POLY_WSUM;  // weight sums: pairs in every 8 on the FMA pipe
 
 // Bounded wait that also gives up once another role has given up.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitBound& wb, int code,
@@ -53,8 +63,8 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const W
     if (mbar_try_wait(addr, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(addr, parity)) return true;
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait_sleep(addr, parity, 20000u)) return true;
         if (*abort_flag) return false;
         if (global_ns() - t0 > wb.ns) {
             record_error(wb, code);
@@ -79,20 +89,25 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // ============================================================================
 // SDPA
 // ============================================================================
+// Two CTAs share an SM: each holds Q (one 128-row tile), one K block and one
+// V block in shared memory, and 256 TMEM columns: S (128 fp32 columns; P, bf16
+// packed two per column, overwrites its first 64 after the softmax has read
+// them) and O (d columns). A CTA's own chain QK(j) -> softmax(j) -> PV(j) ->
+// QK(j+1) is serial; the other CTA's MMAs fill the tensor core meanwhile.
 template <int D>
 struct SdpaCfg {
-    static constexpr int KS = 2;                 // K stages
-    static constexpr int VS = 2;                 // V stages
     static constexpr int HALF = 128 * 128;       // bytes of one 128-row x 64-col bf16 box
     static constexpr int TILE = 128 * D * 2;     // one 128-row x d tile
-    static constexpr int PB = 128 * 128 * 2;     // one P buffer (128 x 128 bf16)
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + TILE;
-    static constexpr int OFF_V = OFF_K + KS * TILE;
-    static constexpr int OFF_P = OFF_V + VS * TILE;
-    static constexpr int OFF_BAR = OFF_P + 2 * PB;
-    static constexpr int NBAR = 24;
-    static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+    static constexpr int OFF_K = TILE;
+    static constexpr int OFF_V = 2 * TILE;
+    static constexpr int OFF_BAR = 3 * TILE;
+    static constexpr int NBAR = 12;
+    static constexpr int SMEM_RAW = OFF_BAR + NBAR * 8 + 16 + 1024;
+    // at least ~80 KB so that no more than two CTAs (2 x 256 TMEM columns)
+    // share an SM
+    static constexpr int SMEM = SMEM_RAW > 80 * 1024 ? SMEM_RAW : 80 * 1024;
+    static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, D, true);
 };
@@ -108,26 +123,23 @@ struct SdpaParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kc,
                const __grid_constant__ CUtensorMap map_vc, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const SdpaParams p) {
     using Cfg = SdpaCfg<D>;
-    constexpr int KS = Cfg::KS, VS = Cfg::VS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* k_full = q_full + 1;
-    uint64_t* k_empty = k_full + KS;
-    uint64_t* v_full = k_empty + KS;
-    uint64_t* v_empty = v_full + VS;
-    uint64_t* s_full = v_empty + VS;
-    uint64_t* s_empty = s_full + 2;
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* pv_done = p_full + 2;
-    uint64_t* o_full = pv_done + 2;
-    uint64_t* drain = o_full + 1;
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = bars + 2;
+    uint64_t* v_full = bars + 3;
+    uint64_t* v_empty = bars + 4;
+    uint64_t* s_full = bars + 5;
+    uint64_t* p_full = bars + 6;
+    uint64_t* pv_done = bars + 7;
+    uint64_t* drain = bars + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -145,31 +157,23 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < KS; ++s) {
-            mbar_init(k_full + s, 1);
-            mbar_init(k_empty + s, 1);
-        }
-        for (int s = 0; s < VS; ++s) {
-            mbar_init(v_full + s, 1);
-            mbar_init(v_empty + s, 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(s_full + s, 1);
-            mbar_init(s_empty + s, 4);
-            mbar_init(p_full + s, 4);
-            mbar_init(pv_done + s, 1);
-        }
-        mbar_init(o_full, 1);
+        mbar_init(k_full, 1);
+        mbar_init(k_empty, 1);
+        mbar_init(v_full, 1);
+        mbar_init(v_empty, 1);
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tc::tmem_alloc(tmem_slot, 512);
+    if (warp == 1) tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
+    const uint32_t tS = tmem, tO = tmem + 128;
 
     const uint32_t sbase = smem_u32(smem);
     if (warp == 0) {
@@ -178,7 +182,7 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             tc::prefetch_tmap(&map_q);
             tc::prefetch_tmap(&map_kc);
             tc::prefetch_tmap(&map_k);
-            int kcount[KS] = {}, vcount[VS] = {};
+            int nk = 0, nv = 0;
             mbar_arrive_expect_tx(q_full, Cfg::TILE);
             const int qrow = (b * p.Hq + h) * p.T + m0;
             for (int hh = 0; hh < D / 64; ++hh)
@@ -188,77 +192,59 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 const CUtensorMap* mk = cache ? &map_kc : &map_k;
                 const CUtensorMap* mv = cache ? &map_vc : &map_v;
                 const int row = cache ? bg * p.C + 128 * j : bg * p.T + 128 * (j - p.nbc);
-                const int ks = j % KS;
-                if (!wait_bar(k_empty + ks, ((j / KS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(k_full + ks, Cfg::TILE);
+                // K(j) once QK(j-1) has read K(j-1)
+                if (!wait_bar(k_empty, (j & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
+                mbar_arrive_expect_tx(k_full, Cfg::TILE);
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_K + ks * Cfg::TILE + hh * Cfg::HALF, mk, 64 * hh, row,
-                                    k_full + ks);
-                ++kcount[ks];
-                const int vs = j % VS;
-                if (!wait_bar(v_empty + vs, ((j / VS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(v_full + vs, Cfg::TILE);
+                    tc::tma_load_2d(smem + Cfg::OFF_K + hh * Cfg::HALF, mk, 64 * hh, row, k_full);
+                ++nk;
+                // V(j) once PV(j-1) has read V(j-1)
+                if (!wait_bar(v_empty, (j & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
+                mbar_arrive_expect_tx(v_full, Cfg::TILE);
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_V + vs * Cfg::TILE + hh * Cfg::HALF, mv, 64 * hh, row,
-                                    v_full + vs);
-                ++vcount[vs];
+                    tc::tma_load_2d(smem + Cfg::OFF_V + hh * Cfg::HALF, mv, 64 * hh, row, v_full);
+                ++nv;
             }
-            // Every load this CTA issued has landed before the CTA can exit
-            // (immediate in the normal case: the MMA warp consumed them all).
+            // every load issued here has landed before the CTA may exit
             wait_bar(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
-            for (int s = 0; s < KS; ++s)
-                if (kcount[s]) wait_bar(k_full + s, (kcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-            for (int s = 0; s < VS; ++s)
-                if (vcount[s]) wait_bar(v_full + s, (vcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            if (nk) wait_bar(k_full, (nk - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            if (nv) wait_bar(v_full, (nv - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------- MMA issuer
         bool ok = warp_wait(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
-        const uint32_t sQ = sbase + Cfg::OFF_Q;
-        for (int j = 0; ok && j <= nb; ++j) {
-            if (j < nb) {
-                const int ks = j % KS, sb = j & 1;
-                ok = warp_wait(k_full + ks, (j / KS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
-                     warp_wait(s_empty + sb, ((j >> 1) & 1) ^ 1, p.wb, kDevTimeoutMmaWait, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t sK = sbase + Cfg::OFF_K + ks * Cfg::TILE;
-                    const uint32_t dS = sb ? tS1 : tS0;
+        const uint32_t sQ = sbase + Cfg::OFF_Q, sK = sbase + Cfg::OFF_K, sV = sbase + Cfg::OFF_V;
+        for (int j = 0; ok && j < nb; ++j) {
+            // S/P columns are free (and O stable) once PV(j-1) has completed
+            ok = warp_wait(k_full, j & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
+                 (j == 0 || warp_wait(pv_done, (j - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag));
+            if (!ok) break;
+            fence_after_sync();
+            if (lane == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-                        tc::mma_bf16_ss(dS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off),
-                                        Cfg::IDESC_QK, kk > 0);
-                    }
-                    tc::mma_commit(s_full + sb);
-                    tc::mma_commit(k_empty + ks);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off), Cfg::IDESC_QK,
+                                    kk > 0);
                 }
-                __syncwarp();
+                tc::mma_commit(s_full);
+                tc::mma_commit(k_empty);
             }
-            if (j >= 1) {
-                const int i = j - 1, pb = i & 1, vs = i % VS;
-                ok = warp_wait(p_full + pb, (i >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag) &&
-                     warp_wait(v_full + vs, (i / VS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t sP = sbase + Cfg::OFF_P + pb * Cfg::PB;
-                    const uint32_t sV = sbase + Cfg::OFF_V + vs * Cfg::TILE;
+            __syncwarp();
+            ok = warp_wait(p_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag) &&
+                 warp_wait(v_full, j & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            if (!ok) break;
+            fence_after_sync();
+            if (lane == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per instruction
-                        const uint32_t aoff = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-                        const uint32_t boff = kk * 16 * 128;
-                        tc::mma_bf16_ss(tO, desc_kmajor_sw128(sP + aoff),
-                                        desc_mnmajor_sw128(sV + boff, Cfg::HALF), Cfg::IDESC_PV,
-                                        (i > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc::mma_commit(v_empty + vs);
-                    tc::mma_commit(pv_done + pb);
-                    if (i == nb - 1) tc::mma_commit(o_full);
+                for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per instruction
+                    tc::mma_bf16_ts(tO, tS + 8 * kk, desc_mnmajor_sw128(sV + kk * 16 * 128, Cfg::HALF),
+                                    Cfg::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                __syncwarp();
+                tc::mma_commit(pv_done);
+                tc::mma_commit(v_empty);
             }
+            __syncwarp();
         }
         // all MMAs issued here complete before TMEM can be released
         if (lane == 0) tc::mma_commit(drain);
@@ -270,85 +256,49 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int r = quad * 32 + lane;  // row inside the tile = TMEM lane
         const int i = m0 + r;            // query row inside the chunk
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
-            const int sb = j & 1;
-            ok = warp_wait(s_full + sb, (j >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+            ok = warp_wait(s_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
             if (!ok) break;
             fence_after_sync();
-            float x[128];
-            {
-                const uint32_t tS = (sb ? tS1 : tS0) + lane_off;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(tS + 32 * c, v);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(v[e]);
-                }
-                tc::tmem_ld_wait();
-            }
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty + sb);
-
             // visible columns of this row in block j: col < limit
             int limit;
             if (j < p.nbc) {
                 limit = p.n - 128 * j;
             } else {
-                const int t0 = 128 * (j - p.nbc);
-                limit = min(i, p.T - 1) - t0 + 1;
+                limit = min(i, p.T - 1) - 128 * (j - p.nbc) + 1;
             }
-            float rmax = -INFINITY;
-            if (limit >= 128) {
+            // pass 1: maximum of the raw visible scores (the scale is positive)
+            float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    x[c] *= p.scale_log2;
-                    rmax = fmaxf(rmax, x[c]);
-                }
-            } else {
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tc::tmem_ld32(tS + lane_off + 32 * c, v);
+                tc::tmem_ld_wait();
+                if (limit >= 128) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    x[c] = (c < limit) ? x[c] * p.scale_log2 : -INFINITY;
-                    rmax = fmaxf(rmax, x[c]);
+                    for (int e = 0; e < 32; e += 4) {
+                        mx0 = tc::max3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        mx1 = tc::max3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float a0 = (32 * c + e < limit) ? __uint_as_float(v[e]) : -INFINITY;
+                        const float a1 = (32 * c + e + 1 < limit) ? __uint_as_float(v[e + 1]) : -INFINITY;
+                        mx0 = tc::max3(mx0, a0, a1);
+                    }
                 }
             }
-            const float m_new = fmaxf(m_run, rmax);
+            const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * p.scale_log2);
             const bool resc = m_new > m_run + kRescaleThreshold;
             const float m_use = resc ? m_new : m_run;
             const float alpha = resc ? ex2(m_run - m_use) : 1.f;
             const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                x[c] = ex2(x[c] - msub);
-                sum += x[c];
-            }
-            // the P buffer is free once PV(j-2) has completed
-            if (j >= 2) {
-                ok = warp_wait(pv_done + sb, ((j - 2) >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
-                if (!ok) break;
-            }
-            {
-                uint8_t* prow = smem + Cfg::OFF_P + sb * Cfg::PB + r * 128;
-#pragma unroll
-                for (int c8 = 0; c8 < 16; ++c8) {
-                    const int half = c8 >> 3, cc = c8 & 7;
-                    uint4 val;
-                    val.x = tc::pack_bf16(x[8 * c8 + 0], x[8 * c8 + 1]);
-                    val.y = tc::pack_bf16(x[8 * c8 + 2], x[8 * c8 + 3]);
-                    val.z = tc::pack_bf16(x[8 * c8 + 4], x[8 * c8 + 5]);
-                    val.w = tc::pack_bf16(x[8 * c8 + 6], x[8 * c8 + 7]);
-                    *reinterpret_cast<uint4*>(prow + half * Cfg::HALF + ((cc ^ (r & 7)) << 4)) = val;
-                }
-            }
             if (j > 0 && __any_sync(0xffffffffu, resc)) {
-                // rescale O in TMEM once PV(j-1) has landed
-                ok = warp_wait(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
+                // O is stable: QK(j) was only issued after PV(j-1) completed
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];
@@ -358,17 +308,46 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
                     tc::tmem_st32(tO + lane_off + 32 * c, v);
                 }
-                tc::tmem_st_wait();
             }
-            tc::fence_proxy_async_smem();
+            // pass 2: P = 2^(s * scale - m) (bf16) into the first 64 columns
+            const float2 nm2 = make_float2(-msub, -msub);
+            float2 sum2 = make_float2(0.f, 0.f), sum2b = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tc::tmem_ld32(tS + lane_off + 32 * c, v);
+                tc::tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float2 x = tc::ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scale2, nm2);
+                    float2 pe;
+                    if (((e >> 1) & 3) < kPolyPairsOf4Sdpa) {
+                        pe = tc::exp2_poly3_x2_ftz(x);
+                    } else {
+                        pe.x = ex2(x.x);
+                        pe.y = ex2(x.y);
+                    }
+                    if (limit < 128) {
+                        pe.x = (32 * c + e < limit) ? pe.x : 0.f;
+                        pe.y = (32 * c + e + 1 < limit) ? pe.y : 0.f;
+                    }
+                    if ((e >> 1) & 1) sum2b = tc::fadd2_ftz(sum2b, pe);
+                    else sum2 = tc::fadd2_ftz(sum2, pe);
+                    pk[e >> 1] = tc::pack_bf16(pe.x, pe.y);
+                }
+                tc::tmem_st16(tS + lane_off + 16 * c, pk);
+            }
+            tc::tmem_st_wait();
             fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + sb);
+            if (lane == 0) mbar_arrive(p_full);
+            const float sum = (sum2.x + sum2.y) + (sum2b.x + sum2b.y);
             l_run = l_run * alpha + sum;
             m_run = m_use;
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && warp_wait(o_full, 0, p.wb, kDevTimeoutMmaWait, abort_flag)) {
+        if (ok && warp_wait(pv_done, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
             fence_after_sync();
             const float inv = 1.f / l_run;
             __nv_bfloat16* orow = p.out + ((size_t)(b * p.Hq + h) * p.T + i) * D;
@@ -396,7 +375,7 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     __syncthreads();
     if (warp == 1) {
         fence_after_sync();
-        tc::tmem_dealloc(tmem, 512);
+        tc::tmem_dealloc(tmem, Cfg::TMEM_COLS);
     }
 }
 
@@ -410,8 +389,8 @@ struct WsumCfg {
     static constexpr int TILE = 128 * D * 2;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_Q = OFF_K + TILE;
-    static constexpr int OFF_ROW = OFF_Q + QS * TILE;     // 2 x 128 x (float lse2, int row)
-    static constexpr int OFF_BAR = OFF_ROW + 2 * 128 * 8;
+    static constexpr int OFF_ROW = OFF_Q + QS * TILE;     // part's rows x (float -lse2, int row)
+    static constexpr int OFF_BAR = OFF_ROW + kRowsPerPart * 8;
     static constexpr int NBAR = 16;
     // at least ~80 KB so that no more than two CTAs (2 x 256 TMEM columns)
     // share an SM
@@ -454,11 +433,11 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     uint64_t* s_full = q_empty + QS;
     uint64_t* s_empty = s_full + 2;
     uint64_t* drain = s_empty + 2;
-    uint64_t* rows_ready = drain + 1;  // [2], 128 arrivals each
+    uint64_t* rows_ready = drain + 1;  // 128 arrivals: the part's row table is in place
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* row_l2 = reinterpret_cast<float*>(smem + Cfg::OFF_ROW);          // [2][128]
-    int* row_i = reinterpret_cast<int*>(smem + Cfg::OFF_ROW + 2 * 128 * 4);  // [2][128]
+    float* row_l2 = reinterpret_cast<float*>(smem + Cfg::OFF_ROW);                 // [kRowsPerPart]
+    int* row_i = reinterpret_cast<int*>(smem + Cfg::OFF_ROW + kRowsPerPart * 4);    // [kRowsPerPart]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     // unit = (key block, row part, group); cache key blocks (most rows) first
@@ -486,8 +465,8 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         for (int s = 0; s < 2; ++s) {
             mbar_init(s_full + s, 1);
             mbar_init(s_empty + s, 4);
-            mbar_init(rows_ready + s, 128);
         }
+        mbar_init(rows_ready, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -558,29 +537,38 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int kr = quad * 32 + lane;       // key row = TMEM lane
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const int t_key = cache ? -1 : t0 + kr;  // chunk token index of this key
-        float acc = 0.f;
-        int cnt = 0;
-        bool ok = true;
-        for (int tt = 0; tt < n_tiles; ++tt) {
-            const int r0 = r_begin + 128 * tt;
-            if (!tile_visible(r0, p.rows_total, p.T, t0)) continue;
-            const int rb = cnt & 1;
-            {   // per-column row data of this tile: log2-domain LSE and chunk row index
-                const int fr = r0 + tid;
-                float l2 = INFINITY;
-                int ii = -1;
+        // the part's row table: minus the log2-domain LSE of each row (-inf
+        // for rows outside the part) and its row index inside the chunk
+        {
+            constexpr int PER = kRowsPerPart / 128;
+            float lv[PER];
+            int iv[PER];
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {  // all loads in flight at once
+                const int fr = r_begin + tid + 128 * q;
+                iv[q] = -1;
+                lv[q] = INFINITY;
                 if (fr < r_end) {
                     const int hh = fr / p.T;
-                    ii = fr - hh * p.T;
-                    l2 = p.lse[(size_t)(qhead0 + hh) * p.tmax + ii] * kLog2e;
+                    iv[q] = fr - hh * p.T;
+                    lv[q] = __ldg(p.lse + (size_t)(qhead0 + hh) * p.tmax + iv[q]);
                 }
-                row_l2[rb * 128 + tid] = l2;
-                row_i[rb * 128 + tid] = ii;
             }
-            mbar_arrive(rows_ready + rb);
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {
+                row_l2[tid + 128 * q] = -lv[q] * kLog2e;
+                row_i[tid + 128 * q] = iv[q];
+            }
+        }
+        mbar_arrive(rows_ready);
+        float acc = 0.f;
+        int cnt = 0;
+        bool ok = warp_wait(rows_ready, 0, p.wb, kDevTimeoutSlotWait, abort_flag);
+        for (int tt = 0; ok && tt < n_tiles; ++tt) {
+            const int r0 = r_begin + 128 * tt;
+            if (!tile_visible(r0, p.rows_total, p.T, t0)) continue;
             const int sb = cnt & 1;
-            ok = warp_wait(rows_ready + rb, (cnt >> 1) & 1, p.wb, kDevTimeoutSlotWait, abort_flag) &&
-                 warp_wait(s_full + sb, (cnt >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+            ok = warp_wait(s_full + sb, (cnt >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
             if (!ok) break;
             fence_after_sync();
             float s[128];
@@ -595,19 +583,49 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_empty + sb);
-            const float* l2 = row_l2 + rb * 128;
-            const int* ri = row_i + rb * 128;
-            float tile_acc = 0.f;
-            if (cache) {
+            const float4* l2v = reinterpret_cast<const float4*>(row_l2 + 128 * tt);
+            const int4* riv = reinterpret_cast<const int4*>(row_i + 128 * tt);
+            // the causal mask matters only for chunk keys on tiles that hold a
+            // row i < t0 + 127 (tiles inside one head starting at i >= t0+127
+            // are fully visible)
+            const int last = min(r0 + 127, r_end - 1);
+            const bool masked = !cache && ((last / p.T != r0 / p.T) || (r0 % p.T) < t0 + 127);
+            const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+            float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
 #pragma unroll
-                for (int c = 0; c < 128; ++c) tile_acc += ex2(fmaf(s[c], p.scale_log2, -l2[c]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const float w = ex2(fmaf(s[c], p.scale_log2, -l2[c]));
-                    tile_acc += (ri[c] >= t_key) ? w : 0.f;
+            for (int c4 = 0; c4 < 32; ++c4) {
+                const float4 L = l2v[c4];
+                float2 w01 = tc::ffma2(make_float2(s[4 * c4], s[4 * c4 + 1]), scale2, make_float2(L.x, L.y));
+                float2 w23 = tc::ffma2(make_float2(s[4 * c4 + 2], s[4 * c4 + 3]), scale2, make_float2(L.z, L.w));
+                const int pair0 = 2 * c4, pair1 = 2 * c4 + 1;
+                if ((pair0 & 7) < kPolyPairsOf8Wsum) {
+                    w01 = tc::exp2_poly3_x2_ftz(w01);
+                } else {
+                    w01.x = ex2(w01.x);
+                    w01.y = ex2(w01.y);
+                }
+                if ((pair1 & 7) < kPolyPairsOf8Wsum) {
+                    w23 = tc::exp2_poly3_x2_ftz(w23);
+                } else {
+                    w23.x = ex2(w23.x);
+                    w23.y = ex2(w23.y);
+                }
+                if (masked) {
+                    const int4 I = riv[c4];
+                    w01.x = (I.x >= t_key) ? w01.x : 0.f;
+                    w01.y = (I.y >= t_key) ? w01.y : 0.f;
+                    w23.x = (I.z >= t_key) ? w23.x : 0.f;
+                    w23.y = (I.w >= t_key) ? w23.y : 0.f;
+                }
+                if (c4 & 1) {
+                    a2 = tc::fadd2_ftz(a2, w01);
+                    a3 = tc::fadd2_ftz(a3, w23);
+                } else {
+                    a0 = tc::fadd2_ftz(a0, w01);
+                    a1 = tc::fadd2_ftz(a1, w23);
                 }
             }
+            const float tile_acc = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
             acc += tile_acc;
             ++cnt;
         }
@@ -620,6 +638,16 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         fence_after_sync();
         tc::tmem_dealloc(tmem, 256);
     }
+}
+
+// Device evaluation of the exp2 variants, for testing them against each other
+// and against a high-precision reference.
+__global__ void exp2_selftest_kernel(const float* x, float* y3, float* y4, float* ym, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    y3[i] = tc::exp2_poly3(x[i]);
+    y4[i] = tc::exp2_poly4(x[i]);
+    ym[i] = ex2(x[i]);
 }
 
 // ============================================================================
@@ -753,6 +781,11 @@ int tc_kernel_plan(int, int, int, int, int, int, int, const char** names, int ma
     const char* plan[2] = {"sdpa_tc_kernel", "wsum_tc_kernel"};
     for (int i = 0; i < 2 && i < max_names; ++i) names[i] = plan[i];
     return 2;
+}
+
+cudaError_t tc_exp2_selftest(const float* x, float* y3, float* y4, float* ym, int n, cudaStream_t s) {
+    exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y3, y4, ym, n);
+    return cudaGetLastError();
 }
 
 cudaError_t tc_sdpa(const StepArgs& a) { return a.d == 64 ? sdpa_launch<64>(a) : sdpa_launch<128>(a); }

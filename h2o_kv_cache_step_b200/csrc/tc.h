@@ -13,6 +13,8 @@ size_t tc_partial_elems(int B, int Hq, int Hkv, int C, int tmax);
 int tc_partial_count(int Hq, int Hkv, int T);
 // Names of the tensor-core kernels one step launches (returns the count).
 int tc_kernel_plan(int B, int Hq, int Hkv, int d, int C, int T, int n, const char** names, int max_names);
+// Evaluates the polynomial exp2 (degrees 3 and 4) and ex2.approx on x[0..n).
+cudaError_t tc_exp2_selftest(const float* x, float* y3, float* y4, float* ym, int n, cudaStream_t s);
 // Chunk SDPA: O and per-row LSE.
 cudaError_t tc_sdpa(const StepArgs& a);
 // Per-key weight sums added to the scores (writes cand_score / cand_pos).

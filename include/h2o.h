@@ -200,6 +200,13 @@ int h2o_select_noalloc(int groups, int C, int n, int T, int64_t P, const float *
                        const int32_t *cand_pos, float *scores, int32_t *positions, uint8_t *kept,
                        int32_t *token_slot, void *stream);
 
+/* Self-test of the exponentials the tensor-core kernels use: for device
+ * float x[0..n), writes the FMA-pipe polynomial 2^x of degree 3 (y_poly3)
+ * and degree 4 (y_poly4), and the hardware approximation ex2.approx.ftz
+ * (y_mufu), all device float [n]. Asynchronous on `stream`. */
+int h2o_selftest_exp2(const float *x, float *y_poly3, float *y_poly4, float *y_mufu, int n,
+                      void *stream);
+
 /* Library build identifier (static string). */
 const char *h2o_version(void);
 

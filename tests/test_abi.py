@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def header_functions():
     src = open(os.path.join(ROOT, "include", "h2o.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(h2o_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(h2o_[a-z_0-9]+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
