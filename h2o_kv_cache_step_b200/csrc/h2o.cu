@@ -56,6 +56,8 @@ struct h2o_ctx {
     int32_t* free_list = nullptr;
     float* partials = nullptr;
     size_t partial_elems = 0;
+    float* nlse2 = nullptr;
+    int rows_pad = 0;
     // host staging for h2o_step_host
     void* stage = nullptr;
     size_t stage_bytes = 0;
@@ -125,6 +127,8 @@ void free_workspace(h2o_ctx* c) {
     cudaFree(c->cand_kept);
     cudaFree(c->token_slot);
     cudaFree(c->partials);
+    cudaFree(c->nlse2);
+    c->nlse2 = nullptr;
     c->lse = c->cand_score = c->partials = nullptr;
     c->cand_pos = c->token_slot = nullptr;
     c->cand_kept = nullptr;
@@ -142,6 +146,8 @@ int alloc_workspace(h2o_ctx* c, int tmax) {
     c->partial_elems = tc_partial_elems(c->B, c->Hq, c->Hkv, c->C, tmax);
     if (c->partial_elems)
         H2O_TRY(c, cudaMalloc(&c->partials, sizeof(float) * c->partial_elems), "cudaMalloc(partials)");
+    c->rows_pad = tc_rows_pad(c->Hq, c->Hkv, tmax);
+    H2O_TRY(c, cudaMalloc(&c->nlse2, sizeof(float) * groups * (size_t)c->rows_pad), "cudaMalloc(nlse2)");
     c->tmax = tmax;
     return H2O_OK;
 }
@@ -187,6 +193,8 @@ StepArgs make_args(h2o_ctx* c, const void* q, const void* k, const void* v, void
     a.free_list = c->free_list;
     a.partials = c->partials;
     a.partial_elems = c->partial_elems;
+    a.nlse2 = c->nlse2;
+    a.rows_pad = c->rows_pad;
     a.wb.err_word = c->err_dev;
     a.wb.ns = c->wait_ns;
     a.stream = s;

@@ -38,6 +38,8 @@ struct StepArgs {
     float* scores;    // [B,Hkv,C]
     int32_t* pos;     // [B,Hkv,C]
     float* lse;       // [B,Hq,tmax] natural-log normaliser per row
+    float* nlse2;     // [B*Hkv, rows_pad] -log2 normaliser per flattened group row (tensor-core path)
+    int rows_pad;
     float* cand_score;   // [B,Hkv,C+tmax]
     int32_t* cand_pos;   // [B,Hkv,C+tmax]
     uint8_t* cand_kept;  // [B,Hkv,C+tmax]

@@ -43,12 +43,14 @@ using tc::fence_after_sync;
 using tc::fence_before_sync;
 
 constexpr int kThreads = 192;
-constexpr int kRowsPerPart = 1024;   // weight-sum rows per CTA (8 tiles of 128)
-constexpr float kRescaleThreshold = 8.f;  // log2 units
+// P may exceed 1 by up to 2^16 before the running maximum is moved: P is
+// bf16 (same exponent range as fp32) and O and the row sum accumulate in fp32,
+// so only overflow matters, and this keeps far from it.
+constexpr float kRescaleThreshold = 16.f;  // log2 units
 // Of every 8 columns, how many take the FMA-pipe exp2 instead of the MUFU
 // unit (the MUFU is the other bottleneck next to the tensor core).
 #ifndef H2O_POLY_SDPA
-#define H2O_POLY_SDPA 1
+#define H2O_POLY_SDPA 0
 #endif
 #ifndef H2O_POLY_WSUM
 #define H2O_POLY_WSUM 2
@@ -89,25 +91,33 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // ============================================================================
 // SDPA
 // ============================================================================
-// Two CTAs share an SM: each holds Q (one 128-row tile), one K block and one
-// V block in shared memory, and 256 TMEM columns: S (128 fp32 columns; P, bf16
-// packed two per column, overwrites its first 64 after the softmax has read
-// them) and O (d columns). A CTA's own chain QK(j) -> softmax(j) -> PV(j) ->
-// QK(j+1) is serial; the other CTA's MMAs fill the tensor core meanwhile.
+// One CTA per SM works on two query tiles at once: rows m0..m0+127 of query
+// heads hA and hB = hA + 1 of the same KV group, so both see the same keys and
+// every K/V block is loaded once for the pair. TMEM (512 columns) holds, per
+// tile, S (128 fp32 columns; P, bf16 packed two per column, overwrites its
+// first 64 after the softmax has read them) and O (d columns). Each tile has
+// its own softmax warpgroup; the MMA warp interleaves the tiles
+//     PV(A,j)  QK(A,j+1)  PV(B,j)  QK(B,j+1)  PV(A,j+1) ...
+// so that one tile's softmax runs while the tensor core works for the other.
+// A group with an odd number of query heads leaves one single-tile CTA per
+// (group, row tile).
 template <int D>
 struct SdpaCfg {
     static constexpr int HALF = 128 * 128;       // bytes of one 128-row x 64-col bf16 box
     static constexpr int TILE = 128 * D * 2;     // one 128-row x d tile
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = TILE;
-    static constexpr int OFF_V = 2 * TILE;
-    static constexpr int OFF_BAR = 3 * TILE;
-    static constexpr int NBAR = 12;
+    static constexpr int KS = 2;                 // K stages
+    static constexpr int VS = 2;                 // V stages
+    static constexpr int OFF_QA = 0;
+    static constexpr int OFF_QB = TILE;
+    static constexpr int OFF_K = 2 * TILE;
+    static constexpr int OFF_V = OFF_K + KS * TILE;
+    static constexpr int OFF_BAR = OFF_V + VS * TILE;
+    static constexpr int NBAR = 24;
     static constexpr int SMEM_RAW = OFF_BAR + NBAR * 8 + 16 + 1024;
-    // at least ~80 KB so that no more than two CTAs (2 x 256 TMEM columns)
-    // share an SM
-    static constexpr int SMEM = SMEM_RAW > 80 * 1024 ? SMEM_RAW : 80 * 1024;
-    static constexpr uint32_t TMEM_COLS = 256;
+    // more than half of an SM's shared memory, so one CTA (512 TMEM columns) per SM
+    static constexpr int SMEM = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int THREADS = 320;          // producer, MMA, 2 x 4 softmax warps
     static constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, D, true);
 };
@@ -116,54 +126,65 @@ struct SdpaParams {
     int B, Hq, Hkv, T, C, n, tmax;
     int n_mblk;   // query-row tiles per head
     int nbc;      // cache key blocks = ceil(n / 128)
+    int npairs;   // head pairs per KV group = ceil(G / 2)
+    int rows_pad; // row stride of nlse2
     float scale_log2;
     __nv_bfloat16* out;
     float* lse;
+    float* nlse2;  // [groups][rows_pad]: -(log2-domain LSE) per flattened group row
     WaitBound wb;
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(SdpaCfg<D>::THREADS, 1)
 sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kc,
                const __grid_constant__ CUtensorMap map_vc, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const SdpaParams p) {
     using Cfg = SdpaCfg<D>;
+    constexpr int KS = Cfg::KS, VS = Cfg::VS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;
-    uint64_t* k_empty = bars + 2;
-    uint64_t* v_full = bars + 3;
-    uint64_t* v_empty = bars + 4;
-    uint64_t* s_full = bars + 5;
-    uint64_t* p_full = bars + 6;
-    uint64_t* pv_done = bars + 7;
-    uint64_t* drain = bars + 8;
+    uint64_t* k_full = bars + 1;           // [KS]
+    uint64_t* k_empty = k_full + KS;       // [KS]
+    uint64_t* v_full = k_empty + KS;       // [VS]
+    uint64_t* v_empty = v_full + VS;       // [VS]
+    uint64_t* s_full = v_empty + VS;       // [2 tiles]
+    uint64_t* p_full = s_full + 2;         // [2 tiles], 4 arrivals
+    uint64_t* pv_done = p_full + 2;        // [2 tiles]
+    uint64_t* drain = pv_done + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // Tiles in decreasing amount of work: the last query-row tile of each head
-    // sees the most chunk keys, so tiles are issued from the last one down.
-    const int BH = p.B * p.Hq;
-    const int mblk = p.n_mblk - 1 - (int)(blockIdx.x / BH);
-    const int bh = blockIdx.x % BH;
-    const int b = bh / p.Hq, h = bh % p.Hq;
+    // unit = (row tile, KV group, head pair); the last row tiles (most keys) first
     const int G = p.Hq / p.Hkv;
-    const int bg = b * p.Hkv + h / G;
+    const int per_mblk = p.B * p.Hkv * p.npairs;
+    const int mblk = p.n_mblk - 1 - (int)(blockIdx.x / per_mblk);
+    const int rest = blockIdx.x % per_mblk;
+    const int bg = rest / p.npairs, pr = rest % p.npairs;
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int hA = g * G + 2 * pr;
+    const bool hasB = 2 * pr + 1 < G;
     const int m0 = mblk * 128;
     const int nb = p.nbc + mblk + 1;  // cache blocks, then chunk blocks 0..mblk
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        mbar_init(k_full, 1);
-        mbar_init(k_empty, 1);
-        mbar_init(v_full, 1);
-        mbar_init(v_empty, 1);
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
+        for (int s = 0; s < KS; ++s) {
+            mbar_init(k_full + s, 1);
+            mbar_init(k_empty + s, 1);
+        }
+        for (int s = 0; s < VS; ++s) {
+            mbar_init(v_full + s, 1);
+            mbar_init(v_empty + s, 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full + t, 1);
+            mbar_init(p_full + t, 4);
+            mbar_init(pv_done + t, 1);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -173,85 +194,146 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
-
     const uint32_t sbase = smem_u32(smem);
+
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             tc::prefetch_tmap(&map_q);
             tc::prefetch_tmap(&map_kc);
             tc::prefetch_tmap(&map_k);
-            int nk = 0, nv = 0;
-            mbar_arrive_expect_tx(q_full, Cfg::TILE);
-            const int qrow = (b * p.Hq + h) * p.T + m0;
-            for (int hh = 0; hh < D / 64; ++hh)
-                tc::tma_load_2d(smem + Cfg::OFF_Q + hh * Cfg::HALF, &map_q, 64 * hh, qrow, q_full);
+            int kcount[KS] = {}, vcount[VS] = {};
+            mbar_arrive_expect_tx(q_full, Cfg::TILE * (hasB ? 2 : 1));
+            for (int hh = 0; hh < D / 64; ++hh) {
+                tc::tma_load_2d(smem + Cfg::OFF_QA + hh * Cfg::HALF, &map_q, 64 * hh, (b * p.Hq + hA) * p.T + m0,
+                                q_full);
+                if (hasB)
+                    tc::tma_load_2d(smem + Cfg::OFF_QB + hh * Cfg::HALF, &map_q, 64 * hh,
+                                    (b * p.Hq + hA + 1) * p.T + m0, q_full);
+            }
             for (int j = 0; j < nb; ++j) {
                 const bool cache = j < p.nbc;
                 const CUtensorMap* mk = cache ? &map_kc : &map_k;
                 const CUtensorMap* mv = cache ? &map_vc : &map_v;
                 const int row = cache ? bg * p.C + 128 * j : bg * p.T + 128 * (j - p.nbc);
-                // K(j) once QK(j-1) has read K(j-1)
-                if (!wait_bar(k_empty, (j & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(k_full, Cfg::TILE);
+                const int ks = j % KS;
+                if (!wait_bar(k_empty + ks, ((j / KS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
+                mbar_arrive_expect_tx(k_full + ks, Cfg::TILE);
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_K + hh * Cfg::HALF, mk, 64 * hh, row, k_full);
-                ++nk;
-                // V(j) once PV(j-1) has read V(j-1)
-                if (!wait_bar(v_empty, (j & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(v_full, Cfg::TILE);
+                    tc::tma_load_2d(smem + Cfg::OFF_K + ks * Cfg::TILE + hh * Cfg::HALF, mk, 64 * hh, row,
+                                    k_full + ks);
+                ++kcount[ks];
+                const int vs = j % VS;
+                if (!wait_bar(v_empty + vs, ((j / VS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
+                mbar_arrive_expect_tx(v_full + vs, Cfg::TILE);
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_V + hh * Cfg::HALF, mv, 64 * hh, row, v_full);
-                ++nv;
+                    tc::tma_load_2d(smem + Cfg::OFF_V + vs * Cfg::TILE + hh * Cfg::HALF, mv, 64 * hh, row,
+                                    v_full + vs);
+                ++vcount[vs];
             }
             // every load issued here has landed before the CTA may exit
             wait_bar(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
-            if (nk) wait_bar(k_full, (nk - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-            if (nv) wait_bar(v_full, (nv - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            for (int s = 0; s < KS; ++s)
+                if (kcount[s]) wait_bar(k_full + s, (kcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            for (int s = 0; s < VS; ++s)
+                if (vcount[s]) wait_bar(v_full + s, (vcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------- MMA issuer
-        bool ok = warp_wait(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
-        const uint32_t sQ = sbase + Cfg::OFF_Q, sK = sbase + Cfg::OFF_K, sV = sbase + Cfg::OFF_V;
-        for (int j = 0; ok && j < nb; ++j) {
-            // S/P columns are free (and O stable) once PV(j-1) has completed
-            ok = warp_wait(k_full, j & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
-                 (j == 0 || warp_wait(pv_done, (j - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag));
-            if (!ok) break;
+        const uint32_t sQA = sbase + Cfg::OFF_QA, sQB = sbase + Cfg::OFF_QB;
+        const uint32_t tSA = tmem, tOA = tmem + 128, tSB = tmem + 256, tOB = tmem + 384;
+        auto issue_qk = [&](uint32_t dS, uint32_t sQ, int ks) {
+            const uint32_t sK = sbase + Cfg::OFF_K + ks * Cfg::TILE;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
+                tc::mma_bf16_ss(dS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off), Cfg::IDESC_QK, kk > 0);
+            }
+        };
+        auto issue_pv = [&](uint32_t dO, uint32_t tP, int vs, bool first) {
+            const uint32_t sV = sbase + Cfg::OFF_V + vs * Cfg::TILE;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per instruction
+                tc::mma_bf16_ts(dO, tP + 8 * kk, desc_mnmajor_sw128(sV + kk * 16 * 128, Cfg::HALF), Cfg::IDESC_PV,
+                                (!first || kk > 0) ? 1u : 0u);
+        };
+        bool ok = warp_wait(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag) &&
+                  warp_wait(k_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
+        if (ok) {
             fence_after_sync();
             if (lane == 0) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off), Cfg::IDESC_QK,
-                                    kk > 0);
-                }
+                issue_qk(tSA, sQA, 0);
                 tc::mma_commit(s_full);
+                if (hasB) {
+                    issue_qk(tSB, sQB, 0);
+                    tc::mma_commit(s_full + 1);
+                }
                 tc::mma_commit(k_empty);
             }
             __syncwarp();
+        }
+        for (int j = 0; ok && j < nb; ++j) {
+            const int vs = j % VS;
+            const bool more = j + 1 < nb;
+            const int ks = (j + 1) % KS;
+            // tile A: PV(A, j), then QK(A, j + 1) once PV(A, j) has read P_A
             ok = warp_wait(p_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag) &&
-                 warp_wait(v_full, j & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+                 warp_wait(v_full + vs, (j / VS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
             if (!ok) break;
             fence_after_sync();
             if (lane == 0) {
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per instruction
-                    tc::mma_bf16_ts(tO, tS + 8 * kk, desc_mnmajor_sw128(sV + kk * 16 * 128, Cfg::HALF),
-                                    Cfg::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-                }
+                issue_pv(tOA, tSA, vs, j == 0);
                 tc::mma_commit(pv_done);
-                tc::mma_commit(v_empty);
+                if (!hasB) tc::mma_commit(v_empty + vs);
             }
             __syncwarp();
+            if (more) {
+                ok = warp_wait(k_full + ks, ((j + 1) / KS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
+                     warp_wait(pv_done, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                if (!ok) break;
+                fence_after_sync();
+                if (lane == 0) {
+                    issue_qk(tSA, sQA, ks);
+                    tc::mma_commit(s_full);
+                    if (!hasB) tc::mma_commit(k_empty + ks);
+                }
+                __syncwarp();
+            }
+            if (hasB) {
+                ok = warp_wait(p_full + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                if (!ok) break;
+                fence_after_sync();
+                if (lane == 0) {
+                    issue_pv(tOB, tSB, vs, j == 0);
+                    tc::mma_commit(pv_done + 1);
+                    tc::mma_commit(v_empty + vs);
+                }
+                __syncwarp();
+                if (more) {
+                    ok = warp_wait(pv_done + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                    if (!ok) break;
+                    fence_after_sync();
+                    if (lane == 0) {
+                        issue_qk(tSB, sQB, ks);
+                        tc::mma_commit(s_full + 1);
+                        tc::mma_commit(k_empty + ks);
+                    }
+                    __syncwarp();
+                }
+            }
         }
         // all MMAs issued here complete before TMEM can be released
         if (lane == 0) tc::mma_commit(drain);
         __syncwarp();
         warp_wait(drain, 0, p.wb, kDevTimeoutMmaWait, abort_flag);
-    } else {
+    } else if (warp < 6 || hasB) {
         // -------------------------------------------------------------- softmax
+        const int X = warp < 6 ? 0 : 1;     // which tile
+        const int h = hA + X;
+        const uint32_t tS = tmem + 256 * X, tO = tmem + 256 * X + 128;
+        uint64_t* my_s_full = s_full + X;
+        uint64_t* my_p_full = p_full + X;
+        uint64_t* my_pv_done = pv_done + X;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;  // row inside the tile = TMEM lane
         const int i = m0 + r;            // query row inside the chunk
@@ -260,94 +342,118 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
-            ok = warp_wait(s_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+            ok = warp_wait(my_s_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
             if (!ok) break;
             fence_after_sync();
             // visible columns of this row in block j: col < limit
-            int limit;
-            if (j < p.nbc) {
-                limit = p.n - 128 * j;
-            } else {
-                limit = min(i, p.T - 1) - 128 * (j - p.nbc) + 1;
-            }
-            // pass 1: maximum of the raw visible scores (the scale is positive)
-            float mx0 = -INFINITY, mx1 = -INFINITY;
+            const int limit = (j < p.nbc) ? p.n - 128 * j : min(i, p.T - 1) - 128 * (j - p.nbc) + 1;
+            // P = 2^(s * scale - m) for the 128 columns, packed bf16 in registers
+            // until the block is accepted; xmax tracks the largest exponent.
+            uint32_t pk[64];
+            float xmax = -INFINITY;
+            float2 sum2 = make_float2(0.f, 0.f), sum2b = make_float2(0.f, 0.f);
+            auto exp_pass = [&](float msub) {
+                const float2 nm2 = make_float2(-msub, -msub);
+                sum2 = make_float2(0.f, 0.f);
+                sum2b = make_float2(0.f, 0.f);
+                float xm0 = -INFINITY, xm1 = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tc::tmem_ld32(tS + lane_off + 32 * c, v);
-                tc::tmem_ld_wait();
-                if (limit >= 128) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        mx0 = tc::max3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                        mx1 = tc::max3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float a0 = (32 * c + e < limit) ? __uint_as_float(v[e]) : -INFINITY;
-                        const float a1 = (32 * c + e + 1 < limit) ? __uint_as_float(v[e + 1]) : -INFINITY;
-                        mx0 = tc::max3(mx0, a0, a1);
-                    }
-                }
-            }
-            const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * p.scale_log2);
-            const bool resc = m_new > m_run + kRescaleThreshold;
-            const float m_use = resc ? m_new : m_run;
-            const float alpha = resc ? ex2(m_run - m_use) : 1.f;
-            const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-            if (j > 0 && __any_sync(0xffffffffu, resc)) {
-                // O is stable: QK(j) was only issued after PV(j-1) completed
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(tO + lane_off + 32 * c, v);
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t v[2][32];
+                    tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
+                    tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                    tc::tmem_st32(tO + lane_off + 32 * c, v);
+                    for (int hv = 0; hv < 2; ++hv) {
+                        const int cbase = 64 * c2 + 32 * hv;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float2 x = tc::ffma2(make_float2(__uint_as_float(v[hv][e]), __uint_as_float(v[hv][e + 1])),
+                                                 scale2, nm2);
+                            if (limit < 128) {
+                                x.x = (cbase + e < limit) ? x.x : -INFINITY;
+                                x.y = (cbase + e + 1 < limit) ? x.y : -INFINITY;
+                            }
+                            if ((e >> 1) & 1) xm1 = tc::max3(xm1, x.x, x.y);
+                            else xm0 = tc::max3(xm0, x.x, x.y);
+                            float2 pe;
+                            if (((e >> 1) & 3) < kPolyPairsOf4Sdpa) {
+                                pe = tc::exp2_poly3_x2_ftz(x);
+                            } else {
+                                pe.x = ex2(x.x);
+                                pe.y = ex2(x.y);
+                            }
+                            if ((e >> 1) & 1) sum2b = tc::fadd2_ftz(sum2b, pe);
+                            else sum2 = tc::fadd2_ftz(sum2, pe);
+                            pk[(cbase + e) >> 1] = tc::pack_bf16(pe.x, pe.y);
+                        }
+                    }
+                }
+                xmax = fmaxf(xm0, xm1);
+            };
+            float alpha = 1.f;
+            bool resc = false;
+            if (j == 0) {
+                // first block: the exact row maximum, then the exponentials
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t v[2][32];
+                    tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
+                    tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int hv = 0; hv < 2; ++hv) {
+                        const int cbase = 64 * c2 + 32 * hv;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float a0 = (cbase + e < limit) ? __uint_as_float(v[hv][e]) : -INFINITY;
+                            const float a1 = (cbase + e + 1 < limit) ? __uint_as_float(v[hv][e + 1]) : -INFINITY;
+                            if ((e >> 1) & 1) mx1 = tc::max3(mx1, a0, a1);
+                            else mx0 = tc::max3(mx0, a0, a1);
+                        }
+                    }
+                }
+                m_run = fmaxf(mx0, mx1) * p.scale_log2;  // every row sees key 0 in block 0
+                exp_pass(m_run);
+            } else {
+                // later blocks: exponents against the running maximum; only if
+                // one exceeds it by more than 2^16 is the block redone
+                exp_pass(m_run);
+                resc = xmax > kRescaleThreshold;
+                if (__any_sync(0xffffffffu, resc)) {
+                    const float m_new = resc ? m_run + xmax : m_run;
+                    alpha = resc ? ex2(m_run - m_new) : 1.f;
+                    // O is stable: QK(j) was only issued after PV(j-1) completed
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t v[32];
+                        tc::tmem_ld32(tO + lane_off + 32 * c, v);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                        tc::tmem_st32(tO + lane_off + 32 * c, v);
+                    }
+                    m_run = m_new;
+                    exp_pass(m_run);
                 }
             }
-            // pass 2: P = 2^(s * scale - m) (bf16) into the first 64 columns
-            const float2 nm2 = make_float2(-msub, -msub);
-            float2 sum2 = make_float2(0.f, 0.f), sum2b = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tc::tmem_ld32(tS + lane_off + 32 * c, v);
-                tc::tmem_ld_wait();
-                uint32_t pk[16];
+                uint32_t q16[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float2 x = tc::ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scale2, nm2);
-                    float2 pe;
-                    if (((e >> 1) & 3) < kPolyPairsOf4Sdpa) {
-                        pe = tc::exp2_poly3_x2_ftz(x);
-                    } else {
-                        pe.x = ex2(x.x);
-                        pe.y = ex2(x.y);
-                    }
-                    if (limit < 128) {
-                        pe.x = (32 * c + e < limit) ? pe.x : 0.f;
-                        pe.y = (32 * c + e + 1 < limit) ? pe.y : 0.f;
-                    }
-                    if ((e >> 1) & 1) sum2b = tc::fadd2_ftz(sum2b, pe);
-                    else sum2 = tc::fadd2_ftz(sum2, pe);
-                    pk[e >> 1] = tc::pack_bf16(pe.x, pe.y);
-                }
-                tc::tmem_st16(tS + lane_off + 16 * c, pk);
+                for (int e = 0; e < 16; ++e) q16[e] = pk[16 * c + e];
+                tc::tmem_st16(tS + lane_off + 16 * c, q16);
             }
             tc::tmem_st_wait();
             fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(my_p_full);
             const float sum = (sum2.x + sum2.y) + (sum2b.x + sum2b.y);
             l_run = l_run * alpha + sum;
-            m_run = m_use;
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && warp_wait(pv_done, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
+        if (ok && warp_wait(my_pv_done, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
             fence_after_sync();
             const float inv = 1.f / l_run;
             __nv_bfloat16* orow = p.out + ((size_t)(b * p.Hq + h) * p.T + i) * D;
@@ -368,7 +474,11 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     }
                 }
             }
-            if (i < p.T) p.lse[(size_t)(b * p.Hq + h) * p.tmax + i] = (m_run + log2f(l_run)) * kLn2;
+            if (i < p.T) {
+                const float lse2 = m_run + log2f(l_run);
+                p.lse[(size_t)(b * p.Hq + h) * p.tmax + i] = lse2 * kLn2;
+                p.nlse2[(size_t)bg * p.rows_pad + (size_t)(h - g * G) * p.T + i] = -lse2;
+            }
         }
     }
     fence_before_sync();
@@ -382,44 +492,83 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 // ============================================================================
 // Weight sums
 // ============================================================================
+// Persistent: one CTA per SM walks a static list of units (KV group, 128-key
+// block, 1024-row part) in decreasing amount of work. Per unit it holds the
+// key block (the A operand, M = 128 keys) and the part's row table (-log2 LSE
+// per query row, fetched with one bulk copy), and streams 256-row query tiles
+// (the B operand, N = 256): S^T = K Q^T lands in one of two 256-column TMEM
+// buffers, one key per lane. Two consumer warpgroups take alternate tiles;
+// each thread sums its key's weights exp2(s * scale - lse2) over the tile's
+// columns in registers. Each warpgroup writes its own partial per unit; the
+// selection kernel adds all partials of a key in a fixed order.
+constexpr int kRowsPerUnit = 1024;
+constexpr int kRowTile = 128;
+constexpr int kTilesPerUnit = kRowsPerUnit / kRowTile;
+
 template <int D>
 struct WsumCfg {
-    static constexpr int QS = 2;                 // Q stages
-    static constexpr int HALF = 128 * 128;
+    static constexpr int QS = 2;                   // Q tile stages
+    static constexpr int HALF = 128 * 128;         // 128 rows x 64 cols box
     static constexpr int TILE = 128 * D * 2;
-    static constexpr int OFF_K = 0;
-    static constexpr int OFF_Q = OFF_K + TILE;
-    static constexpr int OFF_ROW = OFF_Q + QS * TILE;     // part's rows x (float -lse2, int row)
-    static constexpr int OFF_BAR = OFF_ROW + kRowsPerPart * 8;
+    static constexpr int OFF_K = 0;                           // key block
+    static constexpr int OFF_Q = OFF_K + TILE;                // [QS] query tiles
+    static constexpr int OFF_ROW = OFF_Q + QS * TILE;         // [2] row tables (-lse2)
+    static constexpr int OFF_BAR = OFF_ROW + 2 * kRowsPerUnit * 4;
     static constexpr int NBAR = 16;
-    // at least ~80 KB so that no more than two CTAs (2 x 256 TMEM columns)
-    // share an SM
-    static constexpr int SMEM_MIN = 80 * 1024;
     static constexpr int SMEM_RAW = OFF_BAR + NBAR * 8 + 16 + 1024;
-    static constexpr int SMEM = SMEM_RAW > SMEM_MIN ? SMEM_RAW : SMEM_MIN;
-    static constexpr uint32_t IDESC = tc::idesc_bf16_f32(128, 128, false);
+    // at least ~80 KB so that no more than two CTAs (2 x 256 TMEM columns) share an SM
+    static constexpr int SMEM = SMEM_RAW > 80 * 1024 ? SMEM_RAW : 80 * 1024;
+    static constexpr int THREADS = 192;                       // producer, MMA, 4 consumer warps
+    static constexpr uint32_t IDESC = tc::idesc_bf16_f32(128, kRowTile, false);
 };
 
 struct WsumParams {
     int B, Hq, Hkv, T, C, n, tmax;
-    int G, rows_total, nparts, nbc, groups;
+    int G, rows_total, n_ru, nbc, nkb, groups, units, rows_pad;
     float scale_log2;
-    const float* lse;
-    float* partials;   // [nparts][groups][C + tmax]
+    const float* nlse2;   // [groups][rows_pad]: -(log2-domain LSE) per flattened row
+    float* partials;      // [n_ru][groups][C + tmax]
     WaitBound wb;
 };
 
-// Whether any row of tile [r0, r0 + 128) of the group's flattened rows
-// (row = head * T + i) sees chunk token t0 or later (rows i >= t0 do).
-__device__ __forceinline__ bool tile_visible(int r0, int rows_total, int T, int t0) {
+struct WsumUnit {
+    int bg, ru, kb;
+    bool cache;
+    int t0, key_row, cand0, n_keys, r_begin, r_end;
+};
+
+__device__ __forceinline__ WsumUnit wsum_unit(const WsumParams& p, int u) {
+    WsumUnit w;
+    w.bg = u % p.groups;
+    w.ru = (u / p.groups) % p.n_ru;
+    w.kb = u / (p.groups * p.n_ru);
+    w.cache = w.kb < p.nbc;
+    w.t0 = w.cache ? 0 : 128 * (w.kb - p.nbc);
+    w.key_row = w.cache ? w.bg * p.C + 128 * w.kb : w.bg * p.T + w.t0;
+    w.cand0 = w.cache ? 128 * w.kb : p.n + w.t0;
+    w.n_keys = w.cache ? min(128, p.n - 128 * w.kb) : min(128, p.T - w.t0);
+    w.r_begin = w.ru * kRowsPerUnit;
+    w.r_end = min(w.r_begin + kRowsPerUnit, p.rows_total);
+    return w;
+}
+
+// Whether any row of the 128-row tile starting at flattened row r0 (row =
+// head * T + i) sees chunk token t0 or later (rows with i >= t0 do).
+__device__ __forceinline__ bool wtile_visible(int r0, int r_end, int T, int t0) {
+    if (r0 >= r_end) return false;
     if (t0 <= 0) return true;
-    const int last = min(r0 + 127, rows_total - 1);
+    const int last = min(r0 + kRowTile - 1, r_end - 1);
     if (last / T > r0 / T) return true;  // the tile holds the end of a head
     return (last % T) >= t0;
 }
 
+// Persistent weight-sum kernel, two CTAs per SM (each 256 TMEM columns: two
+// 128-column S^T buffers). A CTA walks units (KV group, 128-key block,
+// 1024-row part) in decreasing amount of work; per unit it loads the key
+// block once (the A operand, M = 128 keys) and the part's row table with one
+// bulk copy, and streams 128-row query tiles (the B operand, N = 128).
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(WsumCfg<D>::THREADS, 2)
 wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kc,
                const __grid_constant__ CUtensorMap map_k, const WsumParams p) {
     using Cfg = WsumCfg<D>;
@@ -428,45 +577,31 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
     uint64_t* k_full = bars;
-    uint64_t* q_full = k_full + 1;
-    uint64_t* q_empty = q_full + QS;
-    uint64_t* s_full = q_empty + QS;
-    uint64_t* s_empty = s_full + 2;
+    uint64_t* k_empty = bars + 1;
+    uint64_t* r_full = bars + 2;        // [2]
+    uint64_t* r_empty = bars + 4;       // [2], 4 consumer-warp arrivals
+    uint64_t* q_full = bars + 6;        // [QS]
+    uint64_t* q_empty = q_full + QS;    // [QS]
+    uint64_t* s_full = q_empty + QS;    // [2]
+    uint64_t* s_empty = s_full + 2;     // [2], 4 arrivals
     uint64_t* drain = s_empty + 2;
-    uint64_t* rows_ready = drain + 1;  // 128 arrivals: the part's row table is in place
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* row_l2 = reinterpret_cast<float*>(smem + Cfg::OFF_ROW);                 // [kRowsPerPart]
-    int* row_i = reinterpret_cast<int*>(smem + Cfg::OFF_ROW + kRowsPerPart * 4);    // [kRowsPerPart]
-
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // unit = (key block, row part, group); cache key blocks (most rows) first
-    const int u = blockIdx.x;
-    const int bg = u % p.groups;
-    const int part = (u / p.groups) % p.nparts;
-    const int kb = u / (p.groups * p.nparts);
-    const bool cache = kb < p.nbc;
-    const int t0 = cache ? 0 : 128 * (kb - p.nbc);          // first chunk token of the block
-    const int key_row = cache ? bg * p.C + 128 * kb : bg * p.T + t0;
-    const int cand0 = cache ? 128 * kb : p.n + t0;          // candidate index of lane 0
-    const int n_keys = cache ? min(128, p.n - 128 * kb) : min(128, p.T - t0);
-    const int r_begin = part * kRowsPerPart;
-    const int r_end = min(r_begin + kRowsPerPart, p.rows_total);
-    const int n_tiles = r_end > r_begin ? (r_end - r_begin + 127) / 128 : 0;
-    const int b = bg / p.Hkv, g = bg % p.Hkv;
-    const int qhead0 = b * p.Hq + g * p.G;                  // first query head of the group
 
     if (threadIdx.x == 0) {
         mbar_init(k_full, 1);
+        mbar_init(k_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(r_full + s, 1);
+            mbar_init(r_empty + s, 4);
+            mbar_init(s_full + s, 1);
+            mbar_init(s_empty + s, 4);
+        }
         for (int s = 0; s < QS; ++s) {
             mbar_init(q_full + s, 1);
             mbar_init(q_empty + s, 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(s_full + s, 1);
-            mbar_init(s_empty + s, 4);
-        }
-        mbar_init(rows_ready, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -479,158 +614,176 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     const uint32_t sbase = smem_u32(smem);
 
     if (warp == 0) {
+        // ------------------------------------------------------------ producer
         if (lane == 0) {
             tc::prefetch_tmap(&map_q);
-            int qcount[QS] = {};
-            mbar_arrive_expect_tx(k_full, Cfg::TILE);
-            const CUtensorMap* mk = cache ? &map_kc : &map_k;
-            for (int hh = 0; hh < D / 64; ++hh)
-                tc::tma_load_2d(smem + Cfg::OFF_K + hh * Cfg::HALF, mk, 64 * hh, key_row, k_full);
-            int cnt = 0;
-            for (int tt = 0; tt < n_tiles; ++tt) {
-                const int r0 = r_begin + 128 * tt;
-                if (!tile_visible(r0, p.rows_total, p.T, t0)) continue;
-                const int qs = cnt % QS;
-                if (!wait_bar(q_empty + qs, ((cnt / QS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(q_full + qs, Cfg::TILE);
+            int uc = 0, qc = 0;
+            int kn = 0, rn[2] = {0, 0}, qn[QS] = {};
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++uc) {
+                const WsumUnit w = wsum_unit(p, u);
+                const int st = uc & 1;
+                // row table: -lse2 of the unit's rows (rounded up to 16 bytes)
+                if (!(ok = wait_bar(r_empty + st, ((uc >> 1) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag))) break;
+                const uint32_t rbytes = (uint32_t)(((w.r_end - w.r_begin) + 3) & ~3) * 4u;
+                mbar_arrive_expect_tx(r_full + st, rbytes);
+                tc::bulk_load(smem + Cfg::OFF_ROW + st * kRowsPerUnit * 4,
+                              p.nlse2 + (size_t)w.bg * p.rows_pad + w.r_begin, rbytes, r_full + st);
+                ++rn[st];
+                // key block, once the previous unit's MMAs are done with it
+                if (!(ok = wait_bar(k_empty, (uc & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag))) break;
+                mbar_arrive_expect_tx(k_full, Cfg::TILE);
+                const CUtensorMap* mk = w.cache ? &map_kc : &map_k;
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_Q + qs * Cfg::TILE + hh * Cfg::HALF, &map_q, 64 * hh,
-                                    qhead0 * p.T + r0, q_full + qs);
-                ++qcount[qs];
-                ++cnt;
+                    tc::tma_load_2d(smem + Cfg::OFF_K + hh * Cfg::HALF, mk, 64 * hh, w.key_row, k_full);
+                ++kn;
+                // query tiles
+                const int b = w.bg / p.Hkv, g = w.bg % p.Hkv;
+                const int qrow0 = (b * p.Hq + g * p.G) * p.T;
+                for (int tt = 0; tt < kTilesPerUnit; ++tt) {
+                    const int r0 = w.r_begin + kRowTile * tt;
+                    if (!wtile_visible(r0, w.r_end, p.T, w.t0)) continue;
+                    const int qs = qc % QS;
+                    if (!(ok = wait_bar(q_empty + qs, ((qc / QS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)))
+                        break;
+                    mbar_arrive_expect_tx(q_full + qs, Cfg::TILE);
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        tc::tma_load_2d(smem + Cfg::OFF_Q + qs * Cfg::TILE + hh * Cfg::HALF, &map_q, 64 * hh,
+                                        qrow0 + r0, q_full + qs);
+                    ++qn[qs];
+                    ++qc;
+                }
             }
-            wait_bar(k_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
+            // every load issued here has landed before the CTA may exit
+            if (kn) wait_bar(k_full, (kn - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            for (int s = 0; s < 2; ++s)
+                if (rn[s]) wait_bar(r_full + s, (rn[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
             for (int s = 0; s < QS; ++s)
-                if (qcount[s]) wait_bar(q_full + s, (qcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+                if (qn[s]) wait_bar(q_full + s, (qn[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
         }
     } else if (warp == 1) {
-        bool ok = warp_wait(k_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
+        // ----------------------------------------------------------- MMA issuer
+        int uc = 0, qc = 0, tc_ = 0;
+        bool ok = true;
         const uint32_t sK = sbase + Cfg::OFF_K;
-        int cnt = 0;
-        for (int tt = 0; ok && tt < n_tiles; ++tt) {
-            if (!tile_visible(r_begin + 128 * tt, p.rows_total, p.T, t0)) continue;
-            const int qs = cnt % QS, sb = cnt & 1;
-            ok = warp_wait(q_full + qs, (cnt / QS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
-                 warp_wait(s_empty + sb, ((cnt >> 1) & 1) ^ 1, p.wb, kDevTimeoutMmaWait, abort_flag);
-            if (!ok) break;
-            fence_after_sync();
-            if (lane == 0) {
-                const uint32_t sQ = sbase + Cfg::OFF_Q + qs * Cfg::TILE;
+        for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++uc) {
+            const WsumUnit w = wsum_unit(p, u);
+            if (!(ok = warp_wait(k_full, uc & 1, p.wb, kDevTimeoutTmaWait, abort_flag))) break;
+            for (int tt = 0; tt < kTilesPerUnit; ++tt) {
+                if (!wtile_visible(w.r_begin + kRowTile * tt, w.r_end, p.T, w.t0)) continue;
+                const int qs = qc % QS, sb = tc_ & 1;
+                ok = warp_wait(q_full + qs, (qc / QS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
+                     warp_wait(s_empty + sb, ((tc_ >> 1) & 1) ^ 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                if (!ok) break;
+                fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t sQ = sbase + Cfg::OFF_Q + qs * Cfg::TILE;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tmem + 128 * sb, desc_kmajor_sw128(sK + off), desc_kmajor_sw128(sQ + off),
-                                    Cfg::IDESC, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
+                        tc::mma_bf16_ss(tmem + 128 * sb, desc_kmajor_sw128(sK + off), desc_kmajor_sw128(sQ + off),
+                                        Cfg::IDESC, kk > 0);
+                    }
+                    tc::mma_commit(s_full + sb);
+                    tc::mma_commit(q_empty + qs);
                 }
-                tc::mma_commit(s_full + sb);
-                tc::mma_commit(q_empty + qs);
+                __syncwarp();
+                ++qc;
+                ++tc_;
             }
+            if (!ok) break;
+            if (lane == 0) tc::mma_commit(k_empty);  // after the unit's last MMA
             __syncwarp();
-            ++cnt;
         }
         if (lane == 0) tc::mma_commit(drain);
         __syncwarp();
         warp_wait(drain, 0, p.wb, kDevTimeoutMmaWait, abort_flag);
     } else {
+        // ------------------------------------------------------------ consumers
         const int quad = warp & 3;
-        const int tid = threadIdx.x - 64;      // 0..127: column helper index
-        const int kr = quad * 32 + lane;       // key row = TMEM lane
+        const int kr = quad * 32 + lane;         // key row = TMEM lane
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int t_key = cache ? -1 : t0 + kr;  // chunk token index of this key
-        // the part's row table: minus the log2-domain LSE of each row (-inf
-        // for rows outside the part) and its row index inside the chunk
-        {
-            constexpr int PER = kRowsPerPart / 128;
-            float lv[PER];
-            int iv[PER];
+        int uc = 0, tc_ = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++uc) {
+            const WsumUnit w = wsum_unit(p, u);
+            const int st = uc & 1;
+            if (!(ok = warp_wait(r_full + st, (uc >> 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag))) break;
+            const float* rowt = reinterpret_cast<const float*>(smem + Cfg::OFF_ROW + st * kRowsPerUnit * 4);
+            const int t_key = w.cache ? -1 : w.t0 + kr;  // chunk token index of this key
+            float acc = 0.f;
+            for (int tt = 0; tt < kTilesPerUnit; ++tt) {
+                const int r0 = w.r_begin + kRowTile * tt;
+                if (!wtile_visible(r0, w.r_end, p.T, w.t0)) continue;
+                const int sb = tc_ & 1;
+                const int tcur = tc_++;
+                if (!(ok = warp_wait(s_full + sb, (tcur >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag))) break;
+                fence_after_sync();
+                float s[128];
 #pragma unroll
-            for (int q = 0; q < PER; ++q) {  // all loads in flight at once
-                const int fr = r_begin + tid + 128 * q;
-                iv[q] = -1;
-                lv[q] = INFINITY;
-                if (fr < r_end) {
-                    const int hh = fr / p.T;
-                    iv[q] = fr - hh * p.T;
-                    lv[q] = __ldg(p.lse + (size_t)(qhead0 + hh) * p.tmax + iv[q]);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tc::tmem_ld32(tmem + 128 * sb + lane_off + 32 * c, v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(v[e]);
                 }
-            }
+                tc::tmem_ld_wait();
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_empty + sb);
+                const int ncols = min(kRowTile, w.r_end - r0);  // valid rows in the tile
+                const int last = min(r0 + kRowTile - 1, w.r_end - 1);
+                const bool causal = !w.cache && ((last / p.T != r0 / p.T) || (r0 % p.T) < w.t0 + 127);
+                const float4* rt4 = reinterpret_cast<const float4*>(rowt + kRowTile * tt);
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                if (ncols == kRowTile && !causal) {
 #pragma unroll
-            for (int q = 0; q < PER; ++q) {
-                row_l2[tid + 128 * q] = -lv[q] * kLog2e;
-                row_i[tid + 128 * q] = iv[q];
+                    for (int q4 = 0; q4 < 32; ++q4) {
+                        const float4 L = rt4[q4];
+                        float w0 = fmaf(s[4 * q4 + 0], p.scale_log2, L.x);
+                        float w1 = fmaf(s[4 * q4 + 1], p.scale_log2, L.y);
+                        float w2 = fmaf(s[4 * q4 + 2], p.scale_log2, L.z);
+                        float w3 = fmaf(s[4 * q4 + 3], p.scale_log2, L.w);
+                        if ((q4 & 7) < kPolyPairsOf8Wsum) {
+                            const float2 e01 = tc::exp2_poly3_x2_ftz(make_float2(w0, w1));
+                            const float2 e23 = tc::exp2_poly3_x2_ftz(make_float2(w2, w3));
+                            w0 = e01.x;
+                            w1 = e01.y;
+                            w2 = e23.x;
+                            w3 = e23.y;
+                        } else {
+                            w0 = ex2(w0);
+                            w1 = ex2(w1);
+                            w2 = ex2(w2);
+                            w3 = ex2(w3);
+                        }
+                        // flush-to-zero adds: the polynomial exp2 leaves values
+                        // below 2^-126 as subnormals, which must count as 0
+                        a0 = tc::fadd_ftz(a0, w0);
+                        a1 = tc::fadd_ftz(a1, w1);
+                        a2 = tc::fadd_ftz(a2, w2);
+                        a3 = tc::fadd_ftz(a3, w3);
+                    }
+                } else {
+                    // rows past the part's end, or a causal chunk key: row i
+                    // of column c (i advances with c and wraps at the head end)
+                    int i = r0 % p.T;
+#pragma unroll
+                    for (int c = 0; c < kRowTile; ++c) {
+                        const float wv = ex2(fmaf(s[c], p.scale_log2, rowt[kRowTile * tt + c]));
+                        const bool vis = (c < ncols) && (i >= t_key);
+                        a0 = tc::fadd_ftz(a0, vis ? wv : 0.f);
+                        if (++i == p.T) i = 0;
+                    }
+                }
+                acc += (a0 + a1) + (a2 + a3);
             }
-        }
-        mbar_arrive(rows_ready);
-        float acc = 0.f;
-        int cnt = 0;
-        bool ok = warp_wait(rows_ready, 0, p.wb, kDevTimeoutSlotWait, abort_flag);
-        for (int tt = 0; ok && tt < n_tiles; ++tt) {
-            const int r0 = r_begin + 128 * tt;
-            if (!tile_visible(r0, p.rows_total, p.T, t0)) continue;
-            const int sb = cnt & 1;
-            ok = warp_wait(s_full + sb, (cnt >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
             if (!ok) break;
-            fence_after_sync();
-            float s[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tc::tmem_ld32(tmem + 128 * sb + lane_off + 32 * c, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(v[e]);
-            }
-            tc::tmem_ld_wait();
-            fence_before_sync();
+            if (kr < w.n_keys)
+                p.partials[((size_t)w.ru * p.groups + w.bg) * (size_t)(p.C + p.tmax) + w.cand0 + kr] = acc;
             __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty + sb);
-            const float4* l2v = reinterpret_cast<const float4*>(row_l2 + 128 * tt);
-            const int4* riv = reinterpret_cast<const int4*>(row_i + 128 * tt);
-            // the causal mask matters only for chunk keys on tiles that hold a
-            // row i < t0 + 127 (tiles inside one head starting at i >= t0+127
-            // are fully visible)
-            const int last = min(r0 + 127, r_end - 1);
-            const bool masked = !cache && ((last / p.T != r0 / p.T) || (r0 % p.T) < t0 + 127);
-            const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
-            float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-#pragma unroll
-            for (int c4 = 0; c4 < 32; ++c4) {
-                const float4 L = l2v[c4];
-                float2 w01 = tc::ffma2(make_float2(s[4 * c4], s[4 * c4 + 1]), scale2, make_float2(L.x, L.y));
-                float2 w23 = tc::ffma2(make_float2(s[4 * c4 + 2], s[4 * c4 + 3]), scale2, make_float2(L.z, L.w));
-                const int pair0 = 2 * c4, pair1 = 2 * c4 + 1;
-                if ((pair0 & 7) < kPolyPairsOf8Wsum) {
-                    w01 = tc::exp2_poly3_x2_ftz(w01);
-                } else {
-                    w01.x = ex2(w01.x);
-                    w01.y = ex2(w01.y);
-                }
-                if ((pair1 & 7) < kPolyPairsOf8Wsum) {
-                    w23 = tc::exp2_poly3_x2_ftz(w23);
-                } else {
-                    w23.x = ex2(w23.x);
-                    w23.y = ex2(w23.y);
-                }
-                if (masked) {
-                    const int4 I = riv[c4];
-                    w01.x = (I.x >= t_key) ? w01.x : 0.f;
-                    w01.y = (I.y >= t_key) ? w01.y : 0.f;
-                    w23.x = (I.z >= t_key) ? w23.x : 0.f;
-                    w23.y = (I.w >= t_key) ? w23.y : 0.f;
-                }
-                if (c4 & 1) {
-                    a2 = tc::fadd2_ftz(a2, w01);
-                    a3 = tc::fadd2_ftz(a3, w23);
-                } else {
-                    a0 = tc::fadd2_ftz(a0, w01);
-                    a1 = tc::fadd2_ftz(a1, w23);
-                }
-            }
-            const float tile_acc = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
-            acc += tile_acc;
-            ++cnt;
+            if (lane == 0) mbar_arrive(r_empty + st);
         }
-        if (ok && kr < n_keys)
-            p.partials[((size_t)part * p.groups + bg) * (size_t)(p.C + p.tmax) + cand0 + kr] = acc;
     }
     fence_before_sync();
     __syncthreads();
@@ -670,21 +823,21 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D map over a [rows, d] bf16 matrix, boxes of 128 rows x 64 columns,
+// 2-D map over a [rows, d] bf16 matrix, boxes of box_rows rows x 64 columns,
 // 128-byte swizzle (the layout the UMMA descriptors above describe).
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int nparts_for(int G, int T) { return (G * T + kRowsPerPart - 1) / kRowsPerPart; }
+int nparts_for(int G, int T) { return (G * T + kRowsPerUnit - 1) / kRowsPerUnit; }
 
 template <int D>
 cudaError_t sdpa_launch(const StepArgs& a) {
@@ -710,12 +863,15 @@ cudaError_t sdpa_launch(const StepArgs& a) {
     p.tmax = a.tmax;
     p.n_mblk = (a.T + 127) / 128;
     p.nbc = (a.n + 127) / 128;
+    p.npairs = (a.Hq / a.Hkv + 1) / 2;
+    p.rows_pad = a.rows_pad;
     p.scale_log2 = kLog2e / sqrtf((float)D);
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.lse = a.lse;
+    p.nlse2 = a.nlse2;
     p.wb = a.wb;
-    const int grid = p.n_mblk * a.B * a.Hq;
-    sdpa_tc_kernel<D><<<grid, kThreads, Cfg::SMEM, a.stream>>>(mq, mkc, mvc, mk, mv, p);
+    const int grid = p.n_mblk * a.B * a.Hkv * p.npairs;
+    sdpa_tc_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM, a.stream>>>(mq, mkc, mvc, mk, mv, p);
     a.log->done("sdpa_tc_kernel", a.stream);
     return cudaGetLastError();
 }
@@ -731,11 +887,12 @@ cudaError_t wsum_launch(const StepArgs& a) {
     }
     const int G = a.Hq / a.Hkv;
     const int groups = a.B * a.Hkv;
-    const int nparts = nparts_for(G, a.T);
-    if ((size_t)nparts * groups * (size_t)(a.C + a.tmax) > a.partial_elems) return cudaErrorInvalidValue;
+    const int n_ru = (G * a.T + kRowsPerUnit - 1) / kRowsPerUnit;
+    if ((size_t)n_ru * groups * (size_t)(a.C + a.tmax) > a.partial_elems) return cudaErrorInvalidValue;
     CUtensorMap mq, mkc, mk;
-    if (!make_map(&mq, a.q, (uint64_t)a.B * a.Hq * a.T, D) || !make_map(&mkc, a.Kc, (uint64_t)a.B * a.Hkv * a.C, D) ||
-        !make_map(&mk, a.k, (uint64_t)a.B * a.Hkv * a.T, D))
+    if (!make_map(&mq, a.q, (uint64_t)a.B * a.Hq * a.T, D, kRowTile) ||
+        !make_map(&mkc, a.Kc, (uint64_t)a.B * a.Hkv * a.C, D, 128) ||
+        !make_map(&mk, a.k, (uint64_t)a.B * a.Hkv * a.T, D, 128))
         return cudaErrorInvalidValue;
     WsumParams p;
     p.B = a.B;
@@ -747,16 +904,18 @@ cudaError_t wsum_launch(const StepArgs& a) {
     p.tmax = a.tmax;
     p.G = G;
     p.rows_total = G * a.T;
-    p.nparts = nparts;
+    p.n_ru = n_ru;
     p.nbc = (a.n + 127) / 128;
+    p.nkb = p.nbc + (a.T + 127) / 128;
     p.groups = groups;
+    p.units = p.nkb * n_ru * groups;
+    p.rows_pad = a.rows_pad;
     p.scale_log2 = kLog2e / sqrtf((float)D);
-    p.lse = a.lse;
+    p.nlse2 = a.nlse2;
     p.partials = a.partials;
     p.wb = a.wb;
-    const int nbt = (a.T + 127) / 128;
-    const int grid = (p.nbc + nbt) * nparts * groups;
-    wsum_tc_kernel<D><<<grid, kThreads, Cfg::SMEM, a.stream>>>(mq, mkc, mk, p);
+    const int grid = min(p.units, 2 * a.num_sms);
+    wsum_tc_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM, a.stream>>>(mq, mkc, mk, p);
     a.log->done("wsum_tc_kernel", a.stream);
     return cudaGetLastError();
 }
@@ -773,6 +932,11 @@ bool tc_supported(int device, int d) {
 
 size_t tc_partial_elems(int B, int Hq, int Hkv, int C, int tmax) {
     return (size_t)nparts_for(Hq / Hkv, tmax) * B * Hkv * (size_t)(C + tmax);
+}
+
+int tc_rows_pad(int Hq, int Hkv, int tmax) {
+    const int rows = (Hq / Hkv) * tmax;
+    return (rows + kRowsPerUnit - 1) / kRowsPerUnit * kRowsPerUnit;
 }
 
 int tc_partial_count(int Hq, int Hkv, int T) { return nparts_for(Hq / Hkv, T); }

@@ -9,6 +9,8 @@ namespace h2o {
 bool tc_supported(int device, int d);
 // Workspace floats the weight-sum partials need for chunks of up to tmax tokens.
 size_t tc_partial_elems(int B, int Hq, int Hkv, int C, int tmax);
+// Row stride of the -log2(LSE) table the weight sums read (rows per KV group, padded).
+int tc_rows_pad(int Hq, int Hkv, int tmax);
 // Number of weight-sum partials (row parts) a chunk of T tokens produces.
 int tc_partial_count(int Hq, int Hkv, int T);
 // Names of the tensor-core kernels one step launches (returns the count).
