@@ -36,6 +36,16 @@ __device__ __forceinline__ void record_error(const WaitBound& wb, int code) {
     }
 }
 
+// Programmatic dependent launch: a kernel launched with it may start while
+// the previous kernel on the stream is still finishing; it must call
+// griddep_wait() before touching global memory that earlier work writes or
+// reads. griddep_launch_dependents() lets the next kernel start its own
+// prologue early. Both are no-ops for a normal launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

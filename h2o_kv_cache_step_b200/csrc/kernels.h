@@ -57,6 +57,29 @@ struct StepArgs {
 
 inline int cand_stride(const StepArgs& a) { return a.C + a.tmax; }
 
+// Launch `kernel` on `stream`; with H2O_PDL defined, programmatic dependent
+// launch is allowed (the kernels call griddep_wait() before any global-memory
+// access, so both modes are correct).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+#ifdef H2O_PDL
+    cfg.numAttrs = 1;
+#else
+    cfg.numAttrs = 0;  // measured: no gain for this step's kernel sequence
+#endif
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // SIMT kernels (fp32 path; any supported d).
 cudaError_t launch_sdpa_simt(const StepArgs& a);
 cudaError_t launch_wsum_simt(const StepArgs& a);

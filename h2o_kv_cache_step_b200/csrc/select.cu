@@ -36,7 +36,8 @@ __device__ __forceinline__ uint64_t cand_key(const float* cs, const int32_t* cp,
 
 // Candidate keys are staged in shared memory when they fit (the radix passes
 // then read them from there), otherwise rebuilt from global memory per pass.
-constexpr int kSmemKeyLimit = 24576;  // 192 KB of 64-bit keys
+// The kept flags and the free-slot list always live in shared memory.
+constexpr int kSelectSmemLimit = 220 * 1024;
 
 // Exclusive prefix sum of one int per thread over the block; *total gets the
 // sum. Uses `scratch` (>= 33 ints of shared memory).
@@ -68,6 +69,8 @@ __device__ int block_exclusive_scan(int v, int* scratch, int* total) {
     return r;
 }
 
+// One CTA per (sequence, KV head). Shared memory: the 64-bit candidate keys
+// (when SMEM_KEYS), the kept flags and the free-slot list.
 template <bool SMEM_KEYS>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
@@ -78,36 +81,64 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     __shared__ int scan_scratch[33];
     __shared__ unsigned long long sh_prefix;
     __shared__ int sh_shift, sh_krem, sh_done;
-    extern __shared__ unsigned long long skeys[];  // [m] when SMEM_KEYS
+    extern __shared__ __align__(16) unsigned char dyn[];
 
+    griddep_wait();  // the weight-sum partials are written
+    griddep_launch_dependents();
     const size_t bg = blockIdx.x;
     const int m = n + T;
     float* cs = cand_score + bg * (size_t)(C + tmax);
     int32_t* cp = cand_pos + bg * (size_t)(C + tmax);
-    uint8_t* kept = cand_kept + bg * (size_t)(C + tmax);
-    int32_t* fl = free_list + bg * (size_t)C;
+    uint8_t* kept_g = cand_kept + bg * (size_t)(C + tmax);
     int32_t* ts = token_slot + bg * (size_t)tmax;
     float* sc = scores + bg * (size_t)C;
     int32_t* ps = pos + bg * (size_t)C;
+    // shared layout: [keys m x 8 B (SMEM_KEYS)] [kept m B] [free list C x 4 B]
+    unsigned long long* skeys = reinterpret_cast<unsigned long long*>(dyn);
+    uint8_t* skept = dyn + (SMEM_KEYS ? (size_t)m * 8 : 0);
+    int32_t* sfree = reinterpret_cast<int32_t*>(skept + (((size_t)m + 15) & ~(size_t)15));
 
-    // ---- 0. candidate scores from the weight-sum partials (fixed part order)
-    if (nparts > 0) {
-        const size_t pstride = (size_t)gridDim.x * (C + tmax);
-        for (int c = threadIdx.x; c < m; c += blockDim.x) {
-            float s = c < n ? sc[c] : 0.f;
-            for (int q = 0; q < nparts; ++q) s += partials[q * pstride + bg * (size_t)(C + tmax) + c];
-            cs[c] = s;
-            cp[c] = c < n ? ps[c] : (int32_t)(P + (c - n));
+    // ---- 0. candidate scores (old score + weight-sum partials in a fixed
+    // part order), positions and keys; 4 candidates a thread in flight
+    for (int c0 = threadIdx.x; c0 < m; c0 += 4 * blockDim.x) {
+        float sv[4];
+        int32_t pv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = c0 + u * blockDim.x;
+            sv[u] = 0.f;
+            pv[u] = 0;
+            if (c < m) {
+                if (nparts > 0) {
+                    sv[u] = c < n ? sc[c] : 0.f;
+                    pv[u] = c < n ? ps[c] : (int32_t)(P + (c - n));
+                } else {
+                    sv[u] = cs[c];
+                    pv[u] = cp[c];
+                }
+            }
         }
-        __syncthreads();
+        if (nparts > 0) {
+            const size_t pstride = (size_t)gridDim.x * (C + tmax);
+            for (int q = 0; q < nparts; ++q) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u * blockDim.x;
+                    if (c < m) sv[u] += partials[q * pstride + bg * (size_t)(C + tmax) + c];
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = c0 + u * blockDim.x;
+            if (c >= m) continue;
+            if (nparts > 0) {
+                cs[c] = sv[u];
+                cp[c] = pv[u];
+            }
+            if (SMEM_KEYS) skeys[c] = ((uint64_t)ordered_bits(sv[u]) << 32) | (uint32_t)pv[u];
+        }
     }
-    if (SMEM_KEYS) {
-        for (int c = threadIdx.x; c < m; c += blockDim.x) skeys[c] = cand_key(cs, cp, c);
-        __syncthreads();
-    }
-    auto key_of = [&](int c) -> uint64_t { return SMEM_KEYS ? (uint64_t)skeys[c] : cand_key(cs, cp, c); };
-
-    // ---- 1. threshold: the C-th largest key (radix select, 8 bits a pass)
     if (threadIdx.x == 0) {
         sh_prefix = 0ull;
         sh_shift = 64;
@@ -115,6 +146,10 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         sh_done = (m <= C);
     }
     __syncthreads();
+    auto key_of = [&](int c) -> uint64_t { return SMEM_KEYS ? (uint64_t)skeys[c] : cand_key(cs, cp, c); };
+
+    // ---- 1. threshold: the C-th largest key (MSB-first radix select, 8 bits
+    // a pass, stops as soon as the remaining keys fill one bin exactly)
     while (!sh_done) {
         const int shift = sh_shift - 8;
         const unsigned long long prefix = sh_prefix;
@@ -122,8 +157,7 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         __syncthreads();
         for (int c = threadIdx.x; c < m; c += blockDim.x) {
             const uint64_t key = key_of(c);
-            const bool match = (shift == 56) || ((key >> (shift + 8)) == prefix);
-            if (match) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            if ((shift == 56) || ((key >> (shift + 8)) == prefix)) atomicAdd(&hist[(key >> shift) & 255u], 1u);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -167,11 +201,9 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     // ---- 2. kept flags
     for (int c = threadIdx.x; c < m; c += blockDim.x) {
         bool k = keep_all;
-        if (!keep_all) {
-            const uint64_t key = key_of(c);
-            k = fshift >= 64 ? true : ((key >> fshift) >= fprefix);
-        }
-        kept[c] = (uint8_t)k;
+        if (!keep_all) k = fshift >= 64 ? true : ((key_of(c) >> fshift) >= fprefix);
+        skept[c] = (uint8_t)k;
+        kept_g[c] = (uint8_t)k;
     }
     __syncthreads();
 
@@ -179,11 +211,11 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     const int seg_c = (C + blockDim.x - 1) / blockDim.x;
     const int j0 = min(C, (int)threadIdx.x * seg_c), j1 = min(C, j0 + seg_c);
     int nfree_local = 0;
-    for (int j = j0; j < j1; ++j) nfree_local += (j >= n || !kept[j]);
+    for (int j = j0; j < j1; ++j) nfree_local += (j >= n || !skept[j]);
     int n_free;
     int r = block_exclusive_scan(nfree_local, scan_scratch, &n_free);
     for (int j = j0; j < j1; ++j) {
-        if (j >= n || !kept[j]) fl[r++] = j;
+        if (j >= n || !skept[j]) sfree[r++] = j;
         else sc[j] = cs[j];  // kept cache slot: its updated score
     }
     __syncthreads();
@@ -192,22 +224,22 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     const int seg_t = (T + blockDim.x - 1) / blockDim.x;
     const int t0 = min(T, (int)threadIdx.x * seg_t), t1 = min(T, t0 + seg_t);
     int nk_local = 0;
-    for (int t = t0; t < t1; ++t) nk_local += kept[n + t];
+    for (int t = t0; t < t1; ++t) nk_local += skept[n + t];
     int n_tok;
     int rt = block_exclusive_scan(nk_local, scan_scratch, &n_tok);
     for (int t = t0; t < t1; ++t) {
         int slot = -1;
-        if (kept[n + t] && rt < n_free) {
-            slot = fl[rt];
+        if (skept[n + t] && rt < n_free) {
+            slot = sfree[rt];
             sc[slot] = cs[n + t];
             ps[slot] = (int32_t)(P + t);
         }
-        rt += kept[n + t];
+        rt += skept[n + t];
         ts[t] = slot;
     }
     // free slots nobody took stay (or become) empty
     for (int rr = n_tok + threadIdx.x; rr < n_free; rr += blockDim.x) {
-        const int j = fl[rr];
+        const int j = sfree[rr];
         sc[j] = 0.f;
         ps[j] = -1;
     }
@@ -219,6 +251,8 @@ __global__ void __launch_bounds__(256)
 scatter_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ Kc,
                uint4* __restrict__ Vc, const int32_t* __restrict__ token_slot, int Hkv, int C, int T,
                int tmax, int row_vecs) {
+    griddep_wait();  // the token -> slot map is written
+    griddep_launch_dependents();
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int t = blockIdx.x * 8 + warp;
     const size_t bg = (size_t)blockIdx.z * Hkv + blockIdx.y;
@@ -249,22 +283,30 @@ __global__ void wait_selftest_kernel(WaitBound wb) {
 
 cudaError_t launch_select(const StepArgs& a) {
     const int m = a.n + a.T;
-    if (m <= kSmemKeyLimit) {
-        static int configured = 0;
-        if (!configured) {
-            cudaError_t e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kSmemKeyLimit * 8);
-            if (e != cudaSuccess) return e;
-            configured = 1;
-        }
-        select_kernel<true><<<a.B * a.Hkv, kSelThreads, (size_t)m * 8, a.stream>>>(
-            a.cand_score, a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, a.partials,
-            a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
-    } else {
-        select_kernel<false><<<a.B * a.Hkv, kSelThreads, 0, a.stream>>>(
-            a.cand_score, a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, a.partials,
-            a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
+    const size_t tail = (((size_t)m + 15) & ~(size_t)15) + (size_t)a.C * 4;  // kept flags + free list
+    const size_t with_keys = (size_t)m * 8 + tail;
+    static int configured = 0;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSelectSmemLimit);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmemLimit);
+        if (e != cudaSuccess) return e;
+        configured = 1;
     }
+    cudaError_t e;
+    if (with_keys <= (size_t)kSelectSmemLimit) {
+        e = launch_pdl(select_kernel<true>, dim3(a.B * a.Hkv), dim3(kSelThreads), with_keys, a.stream, a.cand_score,
+                       a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
+                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
+    } else if (tail <= (size_t)kSelectSmemLimit) {
+        e = launch_pdl(select_kernel<false>, dim3(a.B * a.Hkv), dim3(kSelThreads), tail, a.stream, a.cand_score,
+                       a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
+                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
+    } else {
+        return cudaErrorInvalidConfiguration;
+    }
+    if (e != cudaSuccess) return e;
     a.log->done("select_kernel", a.stream);
     return cudaGetLastError();
 }
@@ -273,9 +315,10 @@ cudaError_t launch_scatter(const StepArgs& a) {
     const int elem = a.dtype == 1 ? 4 : 2;
     const int row_vecs = a.d * elem / 16;
     dim3 grid((a.T + 7) / 8, a.Hkv, a.B);
-    scatter_kernel<<<grid, 256, 0, a.stream>>>((const uint4*)a.k, (const uint4*)a.v, (uint4*)a.Kc,
-                                               (uint4*)a.Vc, a.token_slot, a.Hkv, a.C, a.T, a.tmax,
-                                               row_vecs);
+    cudaError_t e = launch_pdl(scatter_kernel, grid, dim3(256), 0, a.stream, (const uint4*)a.k, (const uint4*)a.v,
+                               (uint4*)a.Kc, (uint4*)a.Vc, (const int32_t*)a.token_slot, a.Hkv, a.C, a.T, a.tmax,
+                               row_vecs);
+    if (e != cudaSuccess) return e;
     a.log->done("scatter_kernel", a.stream);
     return cudaGetLastError();
 }

@@ -93,25 +93,27 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // ============================================================================
 // One CTA per SM works on two query tiles at once: rows m0..m0+127 of query
 // heads hA and hB = hA + 1 of the same KV group, so both see the same keys and
-// every K/V block is loaded once for the pair. TMEM (512 columns) holds, per
-// tile, S (128 fp32 columns; P, bf16 packed two per column, overwrites its
-// first 64 after the softmax has read them) and O (d columns). Each tile has
-// its own softmax warpgroup; the MMA warp interleaves the tiles
-//     PV(A,j)  QK(A,j+1)  PV(B,j)  QK(B,j+1)  PV(A,j+1) ...
-// so that one tile's softmax runs while the tensor core works for the other.
+// every K/V block is loaded once for the pair. TMEM (512 columns) holds S and O
+// (128 + d columns) per tile. Each tile has its own softmax warpgroup, which
+// loads S(j) into registers and releases its TMEM columns at once, so QK(j+1)
+// runs on the tensor core while the softmax of block j is still computing;
+// P goes to shared memory (128-byte-swizzled, K-major) for the PV MMA. The
+// tile's serial chain is therefore only its softmax; the tensor core sees
+// QK and PV of both tiles interleaved.
 // A group with an odd number of query heads leaves one single-tile CTA per
 // (group, row tile).
 template <int D>
 struct SdpaCfg {
     static constexpr int HALF = 128 * 128;       // bytes of one 128-row x 64-col bf16 box
     static constexpr int TILE = 128 * D * 2;     // one 128-row x d tile
-    static constexpr int KS = 2;                 // K stages
-    static constexpr int VS = 2;                 // V stages
+    static constexpr int PB = 128 * 128 * 2;     // one P tile (128 rows x 128 keys, bf16)
+    static constexpr int KS = 2;                 // K stages (V has one buffer)
     static constexpr int OFF_QA = 0;
     static constexpr int OFF_QB = TILE;
     static constexpr int OFF_K = 2 * TILE;
     static constexpr int OFF_V = OFF_K + KS * TILE;
-    static constexpr int OFF_BAR = OFF_V + VS * TILE;
+    static constexpr int OFF_P = OFF_V + TILE;   // [2 tiles]
+    static constexpr int OFF_BAR = OFF_P + 2 * PB;
     static constexpr int NBAR = 24;
     static constexpr int SMEM_RAW = OFF_BAR + NBAR * 8 + 16 + 1024;
     // more than half of an SM's shared memory, so one CTA (512 TMEM columns) per SM
@@ -141,17 +143,18 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                const __grid_constant__ CUtensorMap map_vc, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const SdpaParams p) {
     using Cfg = SdpaCfg<D>;
-    constexpr int KS = Cfg::KS, VS = Cfg::VS;
+    constexpr int KS = Cfg::KS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;           // [KS]
     uint64_t* k_empty = k_full + KS;       // [KS]
-    uint64_t* v_full = k_empty + KS;       // [VS]
-    uint64_t* v_empty = v_full + VS;       // [VS]
-    uint64_t* s_full = v_empty + VS;       // [2 tiles]
-    uint64_t* p_full = s_full + 2;         // [2 tiles], 4 arrivals
+    uint64_t* v_full = k_empty + KS;
+    uint64_t* v_empty = v_full + 1;
+    uint64_t* s_full = v_empty + 1;        // [2 tiles]
+    uint64_t* s_free = s_full + 2;         // [2 tiles], 4 arrivals: S loaded into registers
+    uint64_t* p_full = s_free + 2;         // [2 tiles], 4 arrivals: P written to shared memory
     uint64_t* pv_done = p_full + 2;        // [2 tiles]
     uint64_t* drain = pv_done + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
@@ -176,12 +179,11 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
         }
-        for (int s = 0; s < VS; ++s) {
-            mbar_init(v_full + s, 1);
-            mbar_init(v_empty + s, 1);
-        }
+        mbar_init(v_full, 1);
+        mbar_init(v_empty, 1);
         for (int t = 0; t < 2; ++t) {
             mbar_init(s_full + t, 1);
+            mbar_init(s_free + t, 4);
             mbar_init(p_full + t, 4);
             mbar_init(pv_done + t, 1);
         }
@@ -195,14 +197,17 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t sbase = smem_u32(smem);
+    griddep_wait();  // inputs written, and the previous step's readers done
+    griddep_launch_dependents();
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ---------------------------------------------------------- producers
+        // lane 0: Q and the K ring; lane 1: the V buffer (independent waits)
         if (lane == 0) {
             tc::prefetch_tmap(&map_q);
             tc::prefetch_tmap(&map_kc);
             tc::prefetch_tmap(&map_k);
-            int kcount[KS] = {}, vcount[VS] = {};
+            int kcount[KS] = {};
             mbar_arrive_expect_tx(q_full, Cfg::TILE * (hasB ? 2 : 1));
             for (int hh = 0; hh < D / 64; ++hh) {
                 tc::tma_load_2d(smem + Cfg::OFF_QA + hh * Cfg::HALF, &map_q, 64 * hh, (b * p.Hq + hA) * p.T + m0,
@@ -213,34 +218,37 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
             for (int j = 0; j < nb; ++j) {
                 const bool cache = j < p.nbc;
-                const CUtensorMap* mk = cache ? &map_kc : &map_k;
-                const CUtensorMap* mv = cache ? &map_vc : &map_v;
                 const int row = cache ? bg * p.C + 128 * j : bg * p.T + 128 * (j - p.nbc);
                 const int ks = j % KS;
                 if (!wait_bar(k_empty + ks, ((j / KS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
                 mbar_arrive_expect_tx(k_full + ks, Cfg::TILE);
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_K + ks * Cfg::TILE + hh * Cfg::HALF, mk, 64 * hh, row,
-                                    k_full + ks);
+                    tc::tma_load_2d(smem + Cfg::OFF_K + ks * Cfg::TILE + hh * Cfg::HALF, cache ? &map_kc : &map_k,
+                                    64 * hh, row, k_full + ks);
                 ++kcount[ks];
-                const int vs = j % VS;
-                if (!wait_bar(v_empty + vs, ((j / VS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(v_full + vs, Cfg::TILE);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_V + vs * Cfg::TILE + hh * Cfg::HALF, mv, 64 * hh, row,
-                                    v_full + vs);
-                ++vcount[vs];
             }
-            // every load issued here has landed before the CTA may exit
             wait_bar(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
             for (int s = 0; s < KS; ++s)
                 if (kcount[s]) wait_bar(k_full + s, (kcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-            for (int s = 0; s < VS; ++s)
-                if (vcount[s]) wait_bar(v_full + s, (vcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+        } else if (lane == 1) {
+            tc::prefetch_tmap(&map_vc);
+            tc::prefetch_tmap(&map_v);
+            int vcount = 0;
+            for (int j = 0; j < nb; ++j) {
+                const bool cache = j < p.nbc;
+                const int row = cache ? bg * p.C + 128 * j : bg * p.T + 128 * (j - p.nbc);
+                if (!wait_bar(v_empty, (j & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
+                mbar_arrive_expect_tx(v_full, Cfg::TILE);
+                for (int hh = 0; hh < D / 64; ++hh)
+                    tc::tma_load_2d(smem + Cfg::OFF_V + hh * Cfg::HALF, cache ? &map_vc : &map_v, 64 * hh, row,
+                                    v_full);
+                ++vcount;
+            }
+            if (vcount) wait_bar(v_full, (vcount - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------- MMA issuer
-        const uint32_t sQA = sbase + Cfg::OFF_QA, sQB = sbase + Cfg::OFF_QB;
+        const uint32_t sQA = sbase + Cfg::OFF_QA, sQB = sbase + Cfg::OFF_QB, sV = sbase + Cfg::OFF_V;
         const uint32_t tSA = tmem, tOA = tmem + 128, tSB = tmem + 256, tOB = tmem + 384;
         auto issue_qk = [&](uint32_t dS, uint32_t sQ, int ks) {
             const uint32_t sK = sbase + Cfg::OFF_K + ks * Cfg::TILE;
@@ -250,12 +258,14 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 tc::mma_bf16_ss(dS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off), Cfg::IDESC_QK, kk > 0);
             }
         };
-        auto issue_pv = [&](uint32_t dO, uint32_t tP, int vs, bool first) {
-            const uint32_t sV = sbase + Cfg::OFF_V + vs * Cfg::TILE;
+        auto issue_pv = [&](uint32_t dO, int tile, bool first) {
+            const uint32_t sP = sbase + Cfg::OFF_P + tile * Cfg::PB;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per instruction
-                tc::mma_bf16_ts(dO, tP + 8 * kk, desc_mnmajor_sw128(sV + kk * 16 * 128, Cfg::HALF), Cfg::IDESC_PV,
-                                (!first || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per instruction
+                const uint32_t aoff = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
+                tc::mma_bf16_ss(dO, desc_kmajor_sw128(sP + aoff), desc_mnmajor_sw128(sV + kk * 16 * 128, Cfg::HALF),
+                                Cfg::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+            }
         };
         bool ok = warp_wait(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag) &&
                   warp_wait(k_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
@@ -273,54 +283,51 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             __syncwarp();
         }
         for (int j = 0; ok && j < nb; ++j) {
-            const int vs = j % VS;
-            const bool more = j + 1 < nb;
-            const int ks = (j + 1) % KS;
-            // tile A: PV(A, j), then QK(A, j + 1) once PV(A, j) has read P_A
-            ok = warp_wait(p_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag) &&
-                 warp_wait(v_full + vs, (j / VS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-            if (!ok) break;
-            fence_after_sync();
-            if (lane == 0) {
-                issue_pv(tOA, tSA, vs, j == 0);
-                tc::mma_commit(pv_done);
-                if (!hasB) tc::mma_commit(v_empty + vs);
-            }
-            __syncwarp();
-            if (more) {
+            // QK(., j + 1) as soon as each softmax has taken S(j) out of TMEM
+            if (j + 1 < nb) {
+                const int ks = (j + 1) % KS;
                 ok = warp_wait(k_full + ks, ((j + 1) / KS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
-                     warp_wait(pv_done, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                     warp_wait(s_free, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
                 if (!ok) break;
                 fence_after_sync();
                 if (lane == 0) {
                     issue_qk(tSA, sQA, ks);
                     tc::mma_commit(s_full);
-                    if (!hasB) tc::mma_commit(k_empty + ks);
                 }
                 __syncwarp();
-            }
-            if (hasB) {
-                ok = warp_wait(p_full + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
-                if (lane == 0) {
-                    issue_pv(tOB, tSB, vs, j == 0);
-                    tc::mma_commit(pv_done + 1);
-                    tc::mma_commit(v_empty + vs);
-                }
-                __syncwarp();
-                if (more) {
-                    ok = warp_wait(pv_done + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
-                    if (!ok) break;
+                if (hasB) {
+                    if (!(ok = warp_wait(s_free + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag))) break;
                     fence_after_sync();
                     if (lane == 0) {
                         issue_qk(tSB, sQB, ks);
                         tc::mma_commit(s_full + 1);
-                        tc::mma_commit(k_empty + ks);
                     }
                     __syncwarp();
                 }
+                if (lane == 0) tc::mma_commit(k_empty + ks);
+                __syncwarp();
             }
+            // PV(., j) once P(j) is in shared memory
+            ok = warp_wait(p_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag) &&
+                 warp_wait(v_full, j & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            if (!ok) break;
+            fence_after_sync();
+            if (lane == 0) {
+                issue_pv(tOA, 0, j == 0);
+                tc::mma_commit(pv_done);
+            }
+            __syncwarp();
+            if (hasB) {
+                if (!(ok = warp_wait(p_full + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag))) break;
+                fence_after_sync();
+                if (lane == 0) {
+                    issue_pv(tOB, 1, j == 0);
+                    tc::mma_commit(pv_done + 1);
+                }
+                __syncwarp();
+            }
+            if (lane == 0) tc::mma_commit(v_empty);
+            __syncwarp();
         }
         // all MMAs issued here complete before TMEM can be released
         if (lane == 0) tc::mma_commit(drain);
@@ -331,100 +338,50 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int X = warp < 6 ? 0 : 1;     // which tile
         const int h = hA + X;
         const uint32_t tS = tmem + 256 * X, tO = tmem + 256 * X + 128;
-        uint64_t* my_s_full = s_full + X;
-        uint64_t* my_p_full = p_full + X;
-        uint64_t* my_pv_done = pv_done + X;
+        uint8_t* prow_base = smem + Cfg::OFF_P + X * Cfg::PB;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;  // row inside the tile = TMEM lane
         const int i = m0 + r;            // query row inside the chunk
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
-            ok = warp_wait(my_s_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+            ok = warp_wait(s_full + X, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
             if (!ok) break;
             fence_after_sync();
             // visible columns of this row in block j: col < limit
             const int limit = (j < p.nbc) ? p.n - 128 * j : min(i, p.T - 1) - 128 * (j - p.nbc) + 1;
-            // P = 2^(s * scale - m) for the 128 columns, packed bf16 in registers
-            // until the block is accepted; xmax tracks the largest exponent.
-            uint32_t pk[64];
-            float xmax = -INFINITY;
-            float2 sum2 = make_float2(0.f, 0.f), sum2b = make_float2(0.f, 0.f);
-            auto exp_pass = [&](float msub) {
-                const float2 nm2 = make_float2(-msub, -msub);
-                sum2 = make_float2(0.f, 0.f);
-                sum2b = make_float2(0.f, 0.f);
-                float xm0 = -INFINITY, xm1 = -INFINITY;
+            // pass 1 (TMEM): maximum of the raw visible scores (the scale is positive)
+            float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    uint32_t v[2][32];
-                    tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
-                    tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
-                    tc::tmem_ld_wait();
+            for (int c2 = 0; c2 < 2; ++c2) {
+                uint32_t v[2][32];
+                tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
+                tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
+                tc::tmem_ld_wait();
 #pragma unroll
-                    for (int hv = 0; hv < 2; ++hv) {
-                        const int cbase = 64 * c2 + 32 * hv;
+                for (int hv = 0; hv < 2; ++hv) {
+                    const int cbase = 64 * c2 + 32 * hv;
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float2 x = tc::ffma2(make_float2(__uint_as_float(v[hv][e]), __uint_as_float(v[hv][e + 1])),
-                                                 scale2, nm2);
-                            if (limit < 128) {
-                                x.x = (cbase + e < limit) ? x.x : -INFINITY;
-                                x.y = (cbase + e + 1 < limit) ? x.y : -INFINITY;
-                            }
-                            if ((e >> 1) & 1) xm1 = tc::max3(xm1, x.x, x.y);
-                            else xm0 = tc::max3(xm0, x.x, x.y);
-                            float2 pe;
-                            if (((e >> 1) & 3) < kPolyPairsOf4Sdpa) {
-                                pe = tc::exp2_poly3_x2_ftz(x);
-                            } else {
-                                pe.x = ex2(x.x);
-                                pe.y = ex2(x.y);
-                            }
-                            if ((e >> 1) & 1) sum2b = tc::fadd2_ftz(sum2b, pe);
-                            else sum2 = tc::fadd2_ftz(sum2, pe);
-                            pk[(cbase + e) >> 1] = tc::pack_bf16(pe.x, pe.y);
-                        }
+                    for (int e = 0; e < 32; e += 2) {
+                        const float a0 = (cbase + e < limit) ? __uint_as_float(v[hv][e]) : -INFINITY;
+                        const float a1 = (cbase + e + 1 < limit) ? __uint_as_float(v[hv][e + 1]) : -INFINITY;
+                        if ((e >> 1) & 1) mx1 = tc::max3(mx1, a0, a1);
+                        else mx0 = tc::max3(mx0, a0, a1);
                     }
                 }
-                xmax = fmaxf(xm0, xm1);
-            };
-            float alpha = 1.f;
-            bool resc = false;
-            if (j == 0) {
-                // first block: the exact row maximum, then the exponentials
-                float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    uint32_t v[2][32];
-                    tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
-                    tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int hv = 0; hv < 2; ++hv) {
-                        const int cbase = 64 * c2 + 32 * hv;
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const float a0 = (cbase + e < limit) ? __uint_as_float(v[hv][e]) : -INFINITY;
-                            const float a1 = (cbase + e + 1 < limit) ? __uint_as_float(v[hv][e + 1]) : -INFINITY;
-                            if ((e >> 1) & 1) mx1 = tc::max3(mx1, a0, a1);
-                            else mx0 = tc::max3(mx0, a0, a1);
-                        }
-                    }
-                }
-                m_run = fmaxf(mx0, mx1) * p.scale_log2;  // every row sees key 0 in block 0
-                exp_pass(m_run);
-            } else {
-                // later blocks: exponents against the running maximum; only if
-                // one exceeds it by more than 2^16 is the block redone
-                exp_pass(m_run);
-                resc = xmax > kRescaleThreshold;
+            }
+            // the running maximum only moves when it grows by more than 2^16
+            const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * p.scale_log2);
+            const bool resc = m_new > m_run + kRescaleThreshold;
+            const float m_use = resc ? m_new : m_run;
+            const float alpha = resc ? ex2(m_run - m_use) : 1.f;
+            // PV(j-1) has completed: the P buffer is free and O is stable
+            if (j > 0) {
+                ok = warp_wait(pv_done + X, (j - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                if (!ok) break;
+                fence_after_sync();
                 if (__any_sync(0xffffffffu, resc)) {
-                    const float m_new = resc ? m_run + xmax : m_run;
-                    alpha = resc ? ex2(m_run - m_new) : 1.f;
-                    // O is stable: QK(j) was only issued after PV(j-1) completed
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t v[32];
@@ -434,26 +391,59 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                         for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
                         tc::tmem_st32(tO + lane_off + 32 * c, v);
                     }
-                    m_run = m_new;
-                    exp_pass(m_run);
+                    tc::tmem_st_wait();
                 }
             }
+            // pass 2 (TMEM): P = 2^(s * scale - m) -> bf16 -> shared memory; S is
+            // released after its last load so that QK(j+1) can start
+            const float nm = -m_use;
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            uint8_t* prow = prow_base + r * 128;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t q16[16];
+            for (int c2 = 0; c2 < 2; ++c2) {
+                uint32_t v[2][32];
+                tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
+                tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
+                tc::tmem_ld_wait();
+                if (c2 == 1) {
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(s_free + X);
+                }
 #pragma unroll
-                for (int e = 0; e < 16; ++e) q16[e] = pk[16 * c + e];
-                tc::tmem_st16(tS + lane_off + 16 * c, q16);
+                for (int hv = 0; hv < 2; ++hv) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        const int col = 64 * c2 + 32 * hv + 8 * c8;
+                        float e[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            e[k] = ex2(fmaf(__uint_as_float(v[hv][8 * c8 + k]), p.scale_log2, nm));
+                            if (limit < 128) e[k] = (col + k < limit) ? e[k] : 0.f;
+                        }
+                        s0 = tc::fadd_ftz(s0, e[0] + e[4]);
+                        s1 = tc::fadd_ftz(s1, e[1] + e[5]);
+                        s2 = tc::fadd_ftz(s2, e[2] + e[6]);
+                        s3 = tc::fadd_ftz(s3, e[3] + e[7]);
+                        uint4 val;
+                        val.x = tc::pack_bf16(e[0], e[1]);
+                        val.y = tc::pack_bf16(e[2], e[3]);
+                        val.z = tc::pack_bf16(e[4], e[5]);
+                        val.w = tc::pack_bf16(e[6], e[7]);
+                        const int ch = col >> 3, half = ch >> 3, cc = ch & 7;
+                        *reinterpret_cast<uint4*>(prow + half * Cfg::HALF + ((cc ^ (r & 7)) << 4)) = val;
+                    }
+                }
             }
-            tc::tmem_st_wait();
+            tc::fence_proxy_async_smem();
             fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(my_p_full);
-            const float sum = (sum2.x + sum2.y) + (sum2b.x + sum2b.y);
-            l_run = l_run * alpha + sum;
+            if (lane == 0) mbar_arrive(p_full + X);
+            l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
+            m_run = m_use;
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && warp_wait(my_pv_done, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
+        if (ok && warp_wait(pv_done + X, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
             fence_after_sync();
             const float inv = 1.f / l_run;
             __nv_bfloat16* orow = p.out + ((size_t)(b * p.Hq + h) * p.T + i) * D;
@@ -612,6 +602,8 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t sbase = smem_u32(smem);
+    griddep_wait();  // the SDPA's LSE rows are written
+    griddep_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -871,7 +863,9 @@ cudaError_t sdpa_launch(const StepArgs& a) {
     p.nlse2 = a.nlse2;
     p.wb = a.wb;
     const int grid = p.n_mblk * a.B * a.Hkv * p.npairs;
-    sdpa_tc_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM, a.stream>>>(mq, mkc, mvc, mk, mv, p);
+    cudaError_t e = launch_pdl(sdpa_tc_kernel<D>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, a.stream, mq, mkc,
+                               mvc, mk, mv, p);
+    if (e != cudaSuccess) return e;
     a.log->done("sdpa_tc_kernel", a.stream);
     return cudaGetLastError();
 }
@@ -915,7 +909,8 @@ cudaError_t wsum_launch(const StepArgs& a) {
     p.partials = a.partials;
     p.wb = a.wb;
     const int grid = min(p.units, 2 * a.num_sms);
-    wsum_tc_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM, a.stream>>>(mq, mkc, mk, p);
+    cudaError_t e = launch_pdl(wsum_tc_kernel<D>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, a.stream, mq, mkc, mk, p);
+    if (e != cudaSuccess) return e;
     a.log->done("wsum_tc_kernel", a.stream);
     return cudaGetLastError();
 }

@@ -171,6 +171,18 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ---- register reallocation between warpgroups ----------------------------------
+// Executed by all four warps of a warpgroup. The per-thread counts of all
+// warpgroups must add up to at most the registers the block was launched with.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---- misc -------------------------------------------------------------------
 __device__ __forceinline__ float ex2(float x) {
     float y;
