@@ -10,17 +10,19 @@
 //                  the paper page's section "Improvements to Heavy-Hitter
 //                  Oracle (H2O)" adds them to the H2O scores.
 //
-// Both are warp-specialised, one CTA = 6 warps:
-//   warp 0      TMA producer (one elected lane)
-//   warp 1      TMEM owner and tcgen05.mma issuer (one elected lane)
-//   warps 2..5  128 threads, one TMEM lane (matrix row) each
+// Both are warp-specialised: TMA loads and tcgen05.mma issue each have one
+// elected lane of their own warp; 128-thread warpgroups own one TMEM lane
+// (matrix row) per thread.
 //
-// SDPA: M = 128 query rows of one head, N = 128 keys per block, K = d.
-//   S = Q K^T goes to one of two TMEM buffers; the softmax warps turn it into
-//   P (bf16, written to shared memory in the 128-byte-swizzled K-major layout
-//   the next MMA reads) and O += P V accumulates in TMEM. The running maximum
-//   is only moved (and O rescaled in TMEM) when it grows by more than 2^8,
-//   so P stays below 256 and most blocks skip the rescale.
+// SDPA: M = 128 query rows, N = 128 keys per block, K = d; two query tiles
+//   (two heads of one KV group) per CTA, 11 warps: Q/K loader, MMA issuer,
+//   two softmax warpgroups, V loader. S = Q K^T lands in the tile's TMEM
+//   buffer; its softmax warpgroup turns it into P (bf16, written to shared
+//   memory in the 128-byte-swizzled K-major layout the next MMA reads) and
+//   O += P V accumulates in TMEM. The running maximum is only moved (and O
+//   rescaled in TMEM) when it grows by more than 2^16, so most blocks skip the
+//   rescale. One pair of exponentials in every four goes through a degree-3
+//   polynomial on the FMA pipe, the rest through the MUFU unit.
 // Weight sums: the transposed product S^T = K Q^T puts one KEY on each TMEM
 //   lane (M = 128 keys) and 128 query rows on the columns, so each thread sums
 //   its own key's weights across the columns in registers: the reduction over
@@ -50,7 +52,7 @@ constexpr float kRescaleThreshold = 16.f;  // log2 units
 // Of every 8 columns, how many take the FMA-pipe exp2 instead of the MUFU
 // unit (the MUFU is the other bottleneck next to the tensor core).
 #ifndef H2O_POLY_SDPA
-#define H2O_POLY_SDPA 0
+#define H2O_POLY_SDPA 1
 #endif
 #ifndef H2O_POLY_WSUM
 #define H2O_POLY_WSUM 2
@@ -119,7 +121,10 @@ struct SdpaCfg {
     // more than half of an SM's shared memory, so one CTA (512 TMEM columns) per SM
     static constexpr int SMEM = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int THREADS = 320;          // producer, MMA, 2 x 4 softmax warps
+    // warp 0 loads Q and K, warp 1 issues the MMAs, warps 2..9 are the two
+    // softmax warpgroups, warp 10 loads V. The two loaders need warps of their
+    // own: a lane that sleeps in an mbarrier wait suspends its whole warp.
+    static constexpr int THREADS = 352;
     static constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, D, true);
 };
@@ -200,10 +205,10 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     griddep_wait();  // inputs written, and the previous step's readers done
     griddep_launch_dependents();
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 10) {
         // ---------------------------------------------------------- producers
-        // lane 0: Q and the K ring; lane 1: the V buffer (independent waits)
-        if (lane == 0) {
+        // warp 0: Q and the K ring; warp 10: the V buffer
+        if (warp == 0 && lane == 0) {
             tc::prefetch_tmap(&map_q);
             tc::prefetch_tmap(&map_kc);
             tc::prefetch_tmap(&map_k);
@@ -230,7 +235,7 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             wait_bar(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
             for (int s = 0; s < KS; ++s)
                 if (kcount[s]) wait_bar(k_full + s, (kcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-        } else if (lane == 1) {
+        } else if (warp == 10 && lane == 0) {
             tc::prefetch_tmap(&map_vc);
             tc::prefetch_tmap(&map_v);
             int vcount = 0;
@@ -417,9 +422,21 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                         const int col = 64 * c2 + 32 * hv + 8 * c8;
                         float e[8];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            e[k] = ex2(fmaf(__uint_as_float(v[hv][8 * c8 + k]), p.scale_log2, nm));
-                            if (limit < 128) e[k] = (col + k < limit) ? e[k] : 0.f;
+                        for (int k = 0; k < 8; k += 2) {
+                            const float x0 = fmaf(__uint_as_float(v[hv][8 * c8 + k]), p.scale_log2, nm);
+                            const float x1 = fmaf(__uint_as_float(v[hv][8 * c8 + k + 1]), p.scale_log2, nm);
+                            if ((k >> 1) < kPolyPairsOf4Sdpa) {
+                                const float2 pe = tc::exp2_poly3_x2_ftz(make_float2(x0, x1));
+                                e[k] = pe.x;
+                                e[k + 1] = pe.y;
+                            } else {
+                                e[k] = ex2(x0);
+                                e[k + 1] = ex2(x1);
+                            }
+                        }
+                        if (limit < 128) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) e[k] = (col + k < limit) ? e[k] : 0.f;
                         }
                         s0 = tc::fadd_ftz(s0, e[0] + e[4]);
                         s1 = tc::fadd_ftz(s1, e[1] + e[5]);
