@@ -178,6 +178,29 @@ def kernel_work(wl, name: str, n: int, T: int):
     return 0.0, "byte", "hbm"
 
 
+# ------------------------------------------------------------ multi-rank ---
+def rank_workload(wl, rank: int, world: int):
+    """The workload rank `rank` runs: every rank prefills its own sequence
+    (its own seed); the ranks share nothing on the data path."""
+    return wl if world <= 1 else wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest of every rank's x (device timings are taken as the max)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job units per second: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ ours ---
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -186,9 +209,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = synth.WORKLOADS[args.workload]
-    if world > 1:
-        wl = wl.with_(seed=wl.seed + 1000 * rank)  # each rank prefills its own sequence
+    wl = rank_workload(synth.WORKLOADS[args.workload], rank, world)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     sched = sequence_schedule(wl)
 
@@ -260,14 +281,10 @@ def run_ours(args, rank, world, local_rank):
     prof = cache.profile_end()
     cache.sync_check()
 
-    # max over ranks
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_per_step = ms_total / args.steps
-    tokens = (wl.B * wl.N if args.mode == "prefill" else wl.B * wl.T) * args.steps * world
-    value = tokens / (ms_total / 1e3)
+    tokens_per_rank = (wl.B * wl.N if args.mode == "prefill" else wl.B * wl.T) * args.steps
+    value = job_throughput(tokens_per_rank, world, ms_total)
 
     # roofline of the dominant kernel
     peaks, peak_kind = measured_peaks()
@@ -339,12 +356,8 @@ def run_ours(args, rank, world, local_rank):
                 cache.step_host(q, k, v, hout)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": round(wl.B * wl.N * reps * world / (ems / 1e3), 1), "unit": "tokens/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": round(job_throughput(wl.B * wl.N * reps, world, ems), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "h2o_step_host (pinned host buffers, synchronous per chunk)"}
 
