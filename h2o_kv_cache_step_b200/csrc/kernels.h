@@ -57,12 +57,12 @@ struct StepArgs {
 
 inline int cand_stride(const StepArgs& a) { return a.C + a.tmax; }
 
-// Launch `kernel` on `stream`; with H2O_PDL defined, programmatic dependent
-// launch is allowed (the kernels call griddep_wait() before any global-memory
-// access, so both modes are correct).
+// Launch `kernel` on `stream`, allowing programmatic dependent launch if `pdl`
+// (every kernel calls griddep_wait() before it touches global memory that
+// earlier work writes, so both modes are correct).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       Args... args) {
+cudaError_t launch_ex(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -72,12 +72,20 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-#ifdef H2O_PDL
-    cfg.numAttrs = 1;
-#else
-    cfg.numAttrs = 0;  // measured: no gain for this step's kernel sequence
-#endif
+    cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// As launch_ex, with programmatic dependent launch only if H2O_PDL is defined.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+#ifdef H2O_PDL
+    const bool pdl = true;
+#else
+    const bool pdl = false;  // measured: no gain for the tensor-core kernels
+#endif
+    return launch_ex(pdl, kernel, grid, block, smem, stream, args...);
 }
 
 // SIMT kernels (fp32 path; any supported d).

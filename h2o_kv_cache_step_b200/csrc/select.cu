@@ -39,35 +39,39 @@ __device__ __forceinline__ uint64_t cand_key(const float* cs, const int32_t* cp,
 // The kept flags and the free-slot list always live in shared memory.
 constexpr int kSelectSmemLimit = 220 * 1024;
 
-// Exclusive prefix sum of one int per thread over the block; *total gets the
-// sum. Uses `scratch` (>= 33 ints of shared memory).
-__device__ int block_exclusive_scan(int v, int* scratch, int* total) {
+// Exclusive prefix sum of one value per thread over the block; *total gets
+// the sum. Uses `scratch` (>= 33 values of shared memory).
+template <typename V>
+__device__ V block_exclusive_scan(V v, V* scratch, V* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    int x = v;
+    V x = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        const V y = __shfl_up_sync(0xffffffffu, x, off);
         if (lane >= off) x += y;
     }
     if (lane == 31) scratch[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = lane < nwarps ? scratch[lane] : 0;
+        V w = lane < nwarps ? scratch[lane] : V(0);
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, off);
+            const V y = __shfl_up_sync(0xffffffffu, w, off);
             if (lane >= off) w += y;
         }
         if (lane < nwarps) scratch[lane] = w;  // inclusive warp totals
         if (lane == 31) scratch[32] = w;
     }
     __syncthreads();
-    const int base = warp > 0 ? scratch[warp - 1] : 0;
+    const V base = warp > 0 ? scratch[warp - 1] : V(0);
     *total = scratch[32];
-    const int r = base + x - v;
+    const V r = base + x - v;
     __syncthreads();
     return r;
 }
+
+constexpr int kCandPerThread = 4;  // candidates a thread loads per round
+constexpr int kPartBatch = 4;      // weight-sum partials loaded per batch
 
 // One CTA per (sequence, KV head). Shared memory: the 64-bit candidate keys
 // (when SMEM_KEYS), the kept flags and the free-slot list.
@@ -78,15 +82,17 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
               int32_t* __restrict__ free_list, float* __restrict__ scores, int32_t* __restrict__ pos,
               const float* __restrict__ partials, int nparts, int C, int T, int n, int tmax, long long P) {
     __shared__ unsigned int hist[256];
-    __shared__ int scan_scratch[33];
+    __shared__ unsigned long long scan_scratch[33];
+    __shared__ unsigned long long red_min[32], red_max[32];
     __shared__ unsigned long long sh_prefix;
-    __shared__ int sh_shift, sh_krem, sh_done;
+    __shared__ int sh_hi, sh_krem, sh_done;
     extern __shared__ __align__(16) unsigned char dyn[];
 
     griddep_wait();  // the weight-sum partials are written
     griddep_launch_dependents();
     const size_t bg = blockIdx.x;
     const int m = n + T;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float* cs = cand_score + bg * (size_t)(C + tmax);
     int32_t* cp = cand_pos + bg * (size_t)(C + tmax);
     uint8_t* kept_g = cand_kept + bg * (size_t)(C + tmax);
@@ -99,12 +105,14 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     int32_t* sfree = reinterpret_cast<int32_t*>(skept + (((size_t)m + 15) & ~(size_t)15));
 
     // ---- 0. candidate scores (old score + weight-sum partials in a fixed
-    // part order), positions and keys; 4 candidates a thread in flight
-    for (int c0 = threadIdx.x; c0 < m; c0 += 4 * blockDim.x) {
-        float sv[4];
-        int32_t pv[4];
+    // part order), positions and keys; every load of a round is issued
+    // before any is used. Also the smallest and largest key.
+    unsigned long long kmin = ~0ull, kmax = 0ull;
+    for (int c0 = threadIdx.x; c0 < m; c0 += kCandPerThread * blockDim.x) {
+        float sv[kCandPerThread];
+        int32_t pv[kCandPerThread];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kCandPerThread; ++u) {
             const int c = c0 + u * blockDim.x;
             sv[u] = 0.f;
             pv[u] = 0;
@@ -120,49 +128,87 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         }
         if (nparts > 0) {
             const size_t pstride = (size_t)gridDim.x * (C + tmax);
-            for (int q = 0; q < nparts; ++q) {
+            const float* pb = partials + bg * (size_t)(C + tmax);
+            for (int q0 = 0; q0 < nparts; q0 += kPartBatch) {
+                float t[kPartBatch][kCandPerThread];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + u * blockDim.x;
-                    if (c < m) sv[u] += partials[q * pstride + bg * (size_t)(C + tmax) + c];
-                }
+                for (int qq = 0; qq < kPartBatch; ++qq)
+#pragma unroll
+                    for (int u = 0; u < kCandPerThread; ++u) {
+                        const int c = c0 + u * blockDim.x;
+                        t[qq][u] = (q0 + qq < nparts && c < m) ? pb[(size_t)(q0 + qq) * pstride + c] : 0.f;
+                    }
+#pragma unroll
+                for (int qq = 0; qq < kPartBatch; ++qq)
+#pragma unroll
+                    for (int u = 0; u < kCandPerThread; ++u) sv[u] += t[qq][u];  // + 0 for absent parts is exact
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kCandPerThread; ++u) {
             const int c = c0 + u * blockDim.x;
             if (c >= m) continue;
             if (nparts > 0) {
                 cs[c] = sv[u];
                 cp[c] = pv[u];
             }
-            if (SMEM_KEYS) skeys[c] = ((uint64_t)ordered_bits(sv[u]) << 32) | (uint32_t)pv[u];
+            const unsigned long long key = ((uint64_t)ordered_bits(sv[u]) << 32) | (uint32_t)pv[u];
+            if (SMEM_KEYS) skeys[c] = key;
+            kmin = key < kmin ? key : kmin;
+            kmax = key > kmax ? key : kmax;
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, off);
+        const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, off);
+        kmin = a < kmin ? a : kmin;
+        kmax = b > kmax ? b : kmax;
+    }
+    if (lane == 0) {
+        red_min[warp] = kmin;
+        red_max[warp] = kmax;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int nwarps = (int)(blockDim.x >> 5);
+        kmin = lane < nwarps ? red_min[lane] : ~0ull;
+        kmax = lane < nwarps ? red_max[lane] : 0ull;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, off);
+            const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, off);
+            kmin = a < kmin ? a : kmin;
+            kmax = b > kmax ? b : kmax;
         }
     }
     if (threadIdx.x == 0) {
-        sh_prefix = 0ull;
-        sh_shift = 64;
+        // the leading bits every key shares need no radix pass
+        const int common = (m > 0 && kmin != kmax) ? __clzll((long long)(kmin ^ kmax)) : 64;
+        sh_hi = 64 - common;
+        sh_prefix = sh_hi >= 64 ? 0ull : (kmax >> sh_hi);
         sh_krem = C;
-        sh_done = (m <= C);
+        sh_done = (m <= C) || sh_hi == 0;
     }
     __syncthreads();
     auto key_of = [&](int c) -> uint64_t { return SMEM_KEYS ? (uint64_t)skeys[c] : cand_key(cs, cp, c); };
 
-    // ---- 1. threshold: the C-th largest key (MSB-first radix select, 8 bits
-    // a pass, stops as soon as the remaining keys fill one bin exactly)
+    // ---- 1. threshold: the C-th largest key, MSB-first radix select over the
+    // bits below the shared prefix, 8 bits a pass; it stops as soon as the
+    // remaining keys fill one bin exactly
     while (!sh_done) {
-        const int shift = sh_shift - 8;
+        const int hi = sh_hi, lo = hi > 8 ? hi - 8 : 0;
         const unsigned long long prefix = sh_prefix;
+        const unsigned long long dmask = (1ull << (hi - lo)) - 1ull;
         for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0u;
         __syncthreads();
         for (int c = threadIdx.x; c < m; c += blockDim.x) {
             const uint64_t key = key_of(c);
-            if ((shift == 56) || ((key >> (shift + 8)) == prefix)) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            if ((hi >= 64) || ((key >> hi) == prefix)) atomicAdd(&hist[(unsigned int)((key >> lo) & dmask)], 1u);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
             // lane l owns bins 255-8l down to 248-8l (descending key order)
-            const int lane = threadIdx.x;
             unsigned int cnt[8], lsum = 0;
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
@@ -184,36 +230,44 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
                     above += cnt[r];
                     ++r;
                 }
-                const unsigned int digit = 255u - 8u * lane - r;
+                const unsigned long long digit = 255u - 8u * lane - r;
                 const unsigned int new_krem = krem - above;
-                sh_prefix = (prefix << 8) | digit;
-                sh_shift = shift;
+                sh_prefix = (hi >= 64 ? 0ull : (prefix << (hi - lo))) | digit;
+                sh_hi = lo;
                 sh_krem = (int)new_krem;
-                sh_done = (cnt[r] == new_krem) || shift == 0;
+                sh_done = (cnt[r] == new_krem) || lo == 0;
             }
         }
         __syncthreads();
     }
-    const int fshift = sh_shift;
+    const int fhi = sh_hi;
     const unsigned long long fprefix = sh_prefix;
     const bool keep_all = (m <= C);
 
-    // ---- 2. kept flags
+    // ---- 2. kept flags: a key is kept iff its bits above fhi are at least
+    // the threshold's (every key whose leading bits lie above the threshold's,
+    // and the whole final bin)
     for (int c = threadIdx.x; c < m; c += blockDim.x) {
-        bool k = keep_all;
-        if (!keep_all) k = fshift >= 64 ? true : ((key_of(c) >> fshift) >= fprefix);
+        const bool k = keep_all || fhi >= 64 || ((key_of(c) >> fhi) >= fprefix);
         skept[c] = (uint8_t)k;
         kept_g[c] = (uint8_t)k;
     }
     __syncthreads();
 
-    // ---- 3. free slots (empty, or holding an evicted entry), ascending
+    // ---- 3. one scan for both: free slots (empty, or holding an evicted
+    // entry) in ascending order, and kept chunk tokens in position order
     const int seg_c = (C + blockDim.x - 1) / blockDim.x;
     const int j0 = min(C, (int)threadIdx.x * seg_c), j1 = min(C, j0 + seg_c);
-    int nfree_local = 0;
+    const int seg_t = (T + blockDim.x - 1) / blockDim.x;
+    const int t0 = min(T, (int)threadIdx.x * seg_t), t1 = min(T, t0 + seg_t);
+    unsigned long long nfree_local = 0, nk_local = 0;
     for (int j = j0; j < j1; ++j) nfree_local += (j >= n || !skept[j]);
-    int n_free;
-    int r = block_exclusive_scan(nfree_local, scan_scratch, &n_free);
+    for (int t = t0; t < t1; ++t) nk_local += skept[n + t];
+    unsigned long long total;
+    const unsigned long long ex =
+        block_exclusive_scan<unsigned long long>((nfree_local << 32) | nk_local, scan_scratch, &total);
+    const int n_free = (int)(total >> 32), n_tok = (int)(total & 0xffffffffull);
+    int r = (int)(ex >> 32);
     for (int j = j0; j < j1; ++j) {
         if (j >= n || !skept[j]) sfree[r++] = j;
         else sc[j] = cs[j];  // kept cache slot: its updated score
@@ -221,12 +275,7 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     __syncthreads();
 
     // ---- 4. kept chunk tokens, in position order, take the free slots
-    const int seg_t = (T + blockDim.x - 1) / blockDim.x;
-    const int t0 = min(T, (int)threadIdx.x * seg_t), t1 = min(T, t0 + seg_t);
-    int nk_local = 0;
-    for (int t = t0; t < t1; ++t) nk_local += skept[n + t];
-    int n_tok;
-    int rt = block_exclusive_scan(nk_local, scan_scratch, &n_tok);
+    int rt = (int)(ex & 0xffffffffull);
     for (int t = t0; t < t1; ++t) {
         int slot = -1;
         if (skept[n + t] && rt < n_free) {
@@ -281,6 +330,12 @@ __global__ void wait_selftest_kernel(WaitBound wb) {
 
 }  // namespace
 
+// The selection and copy kernels are launched with programmatic dependent
+// launch: their CTAs start (and fetch their code) while the previous kernel
+// drains, then wait for it in griddep_wait(). Measured on the bench's prefill:
+// -3% step time; the same for the SDPA and weight-sum launches measured no gain.
+constexpr bool kEarlyLaunch = true;
+
 cudaError_t launch_select(const StepArgs& a) {
     const int m = a.n + a.T;
     const size_t tail = (((size_t)m + 15) & ~(size_t)15) + (size_t)a.C * 4;  // kept flags + free list
@@ -296,11 +351,11 @@ cudaError_t launch_select(const StepArgs& a) {
     }
     cudaError_t e;
     if (with_keys <= (size_t)kSelectSmemLimit) {
-        e = launch_pdl(select_kernel<true>, dim3(a.B * a.Hkv), dim3(kSelThreads), with_keys, a.stream, a.cand_score,
+        e = launch_ex(kEarlyLaunch, select_kernel<true>, dim3(a.B * a.Hkv), dim3(kSelThreads), with_keys, a.stream, a.cand_score,
                        a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
                        a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
     } else if (tail <= (size_t)kSelectSmemLimit) {
-        e = launch_pdl(select_kernel<false>, dim3(a.B * a.Hkv), dim3(kSelThreads), tail, a.stream, a.cand_score,
+        e = launch_ex(kEarlyLaunch, select_kernel<false>, dim3(a.B * a.Hkv), dim3(kSelThreads), tail, a.stream, a.cand_score,
                        a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
                        a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
     } else {
@@ -315,7 +370,7 @@ cudaError_t launch_scatter(const StepArgs& a) {
     const int elem = a.dtype == 1 ? 4 : 2;
     const int row_vecs = a.d * elem / 16;
     dim3 grid((a.T + 7) / 8, a.Hkv, a.B);
-    cudaError_t e = launch_pdl(scatter_kernel, grid, dim3(256), 0, a.stream, (const uint4*)a.k, (const uint4*)a.v,
+    cudaError_t e = launch_ex(kEarlyLaunch, scatter_kernel, grid, dim3(256), 0, a.stream, (const uint4*)a.k, (const uint4*)a.v,
                                (uint4*)a.Kc, (uint4*)a.Vc, (const int32_t*)a.token_slot, a.Hkv, a.C, a.T, a.tmax,
                                row_vecs);
     if (e != cudaSuccess) return e;
