@@ -334,16 +334,19 @@ def run_ours(args, rank, world, local_rank):
                  "frac_of_measured_burst": round(ach / peaks["bf16_tflops"], 4),
                  "frac_of_spec_2250": round(ach / 2250.0, 4)}
 
-    # end to end through h2o_step_host with pinned host buffers
+    # end to end through the host-buffer API (pinned memory): every chunk's
+    # inputs are uploaded and its output downloaded inside the timed region;
+    # the pipelined call overlaps chunk c's step with the copies of its neighbours
     e2e = None
     if not args.no_e2e and args.mode == "prefill":
         host = [tuple(t.cpu().pin_memory() for t in ch) for ch in chunks]
-        hout = torch.empty_like(chunks[0][0], device="cpu").pin_memory()
+        houts = [torch.empty_like(chunks[0][0], device="cpu").pin_memory() for _ in range(wl.n_chunks)]
         h2d = sum(t.numel() * t.element_size() for ch in host for t in ch)
-        d2h = hout.numel() * hout.element_size() * wl.n_chunks
+        d2h = sum(t.numel() * t.element_size() for t in houts)
         cache.reset()
-        for (q, k, v) in host[:2]:
-            cache.step_host(q, k, v, hout)
+        for (q, k, v), ho in zip(host[:2], houts):
+            cache.step_host_async(q, k, v, ho)
+        cache.host_sync()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -352,14 +355,15 @@ def run_ours(args, rank, world, local_rank):
         e0.record(stream)
         for _ in range(reps):
             cache.reset()
-            for (q, k, v) in host:
-                cache.step_host(q, k, v, hout)
+            for (q, k, v), ho in zip(host, houts):
+                cache.step_host_async(q, k, v, ho)
+            cache.host_sync()  # every output is in host memory
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), dev)
         e2e = {"value": round(job_throughput(wl.B * wl.N * reps, world, ems), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "h2o_step_host (pinned host buffers, synchronous per chunk)"}
+               "api": "h2o_step_host_async + h2o_host_sync (pinned host buffers; uploads, steps and downloads of successive chunks overlap; one host sync per prefill)"}
 
     result = {
         "metric": METRIC,

@@ -38,6 +38,8 @@ SIGNATURES = [
     ("h2o_destroy", _I, [_P]),
     ("h2o_step", _I, [_P, _P, _P, _P, _P, _I, _P]),
     ("h2o_step_host", _I, [_P, _P, _P, _P, _P, _I, _P]),
+    ("h2o_step_host_async", _I, [_P, _P, _P, _P, _P, _I, _P]),
+    ("h2o_host_sync", _I, [_P]),
     ("h2o_scores", _I, [_P, _P, _P]),
     ("h2o_positions", _I, [_P, _P, _P]),
     ("h2o_counters", _I, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),

@@ -76,16 +76,37 @@ class H2OCache:
                                    _stream_ptr(stream)))
         return out
 
+    def _check_host(self, q, k, v, out) -> int:
+        T = q.shape[2]
+        for name, t, heads in (("q", q, self.Hq), ("k", k, self.Hkv), ("v", v, self.Hkv), ("out", out, self.Hq)):
+            if (t.is_cuda or not t.is_contiguous() or t.dtype != self.dtype
+                    or tuple(t.shape) != (self.B, heads, T, self.d)):
+                raise ValueError(f"{name}: need a contiguous host {self.dtype} tensor of shape "
+                                 f"{(self.B, heads, T, self.d)}, got {t.dtype} {tuple(t.shape)}")
+        return T
+
     def step_host(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                   out: torch.Tensor, stream=None) -> torch.Tensor:
-        """Same step on host (CPU) tensors; pinned memory gives async copies."""
-        T = q.shape[2]
-        for t in (q, k, v, out):
-            if t.is_cuda or not t.is_contiguous() or t.dtype != self.dtype:
-                raise ValueError("step_host needs contiguous host tensors of the cache dtype")
+        """Same step on host (CPU) tensors; pinned memory gives async copies.
+        Returns once the output is in `out`."""
+        T = self._check_host(q, k, v, out)
         self._check(lib().h2o_step_host(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), T,
                                         _stream_ptr(stream)))
         return out
+
+    def step_host_async(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                        out: torch.Tensor, stream=None) -> torch.Tensor:
+        """Pipelined step on host tensors (use pinned memory): returns at once;
+        the inputs must stay unchanged and `out` is valid only after
+        host_sync(). Successive chunks overlap copies with the steps."""
+        T = self._check_host(q, k, v, out)
+        self._check(lib().h2o_step_host_async(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), T,
+                                              _stream_ptr(stream)))
+        return out
+
+    def host_sync(self) -> None:
+        """Wait for every step_host_async copy (outputs are then in host memory)."""
+        self._check(lib().h2o_host_sync(self._h))
 
     # -- inspection ---------------------------------------------------------
     def counters(self) -> tuple[int, int]:

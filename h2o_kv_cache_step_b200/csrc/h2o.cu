@@ -61,6 +61,15 @@ struct h2o_ctx {
     // host staging for h2o_step_host
     void* stage = nullptr;
     size_t stage_bytes = 0;
+    // pipelined host path (h2o_step_host_async): two staging slots, an upload
+    // and a download stream, and per-slot events
+    void* aslot[2] = {nullptr, nullptr};
+    size_t aslot_bytes = 0;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_in[2] = {nullptr, nullptr};    // slot's inputs uploaded
+    cudaEvent_t ev_step[2] = {nullptr, nullptr};  // step reading the slot done
+    cudaEvent_t ev_out[2] = {nullptr, nullptr};   // slot's output downloaded
+    long long achunks = 0;
     // error word (host-mapped)
     int* err_host = nullptr;
     int* err_dev = nullptr;
@@ -117,6 +126,24 @@ struct DeviceGuard {
         if (changed) cudaSetDevice(prev);
     }
 };
+
+// Releases the pipelined host path's streams, events and staging slots.
+void free_async(h2o_ctx* c) {
+    if (c->s_in) cudaStreamSynchronize(c->s_in);
+    if (c->s_out) cudaStreamSynchronize(c->s_out);
+    for (int i = 0; i < 2; ++i) {
+        cudaFree(c->aslot[i]);
+        c->aslot[i] = nullptr;
+        for (cudaEvent_t* e : {&c->ev_in[i], &c->ev_step[i], &c->ev_out[i]}) {
+            if (*e) cudaEventDestroy(*e);
+            *e = nullptr;
+        }
+    }
+    if (c->s_in) cudaStreamDestroy(c->s_in);
+    if (c->s_out) cudaStreamDestroy(c->s_out);
+    c->s_in = c->s_out = nullptr;
+    c->aslot_bytes = 0;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -278,6 +305,7 @@ int h2o_destroy(h2o_ctx* c) {
     if (!c) return H2O_OK;
     DeviceGuard g(c->device);
     cudaDeviceSynchronize();
+    free_async(c);
     free_workspace(c);
     for (cudaEvent_t e : c->prof_ev) cudaEventDestroy(e);
     cudaFree(c->Kc);
@@ -399,6 +427,74 @@ int h2o_step_host(h2o_ctx* c, const void* q, const void* k, const void* v, void*
     if (rc != H2O_OK) return rc;
     H2O_TRY(c, cudaMemcpyAsync(out, dout, qb, cudaMemcpyDeviceToHost, s), "copy out to host");
     H2O_TRY(c, cudaStreamSynchronize(s), "synchronise after step");
+    return check_ctx(c);
+}
+
+
+int h2o_step_host_async(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T,
+                        void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (T < 1) return fail(c, H2O_ERR_ARG, "T must be >= 1 (got %d)", T);
+    if (!q || !k || !v || !out) return fail(c, H2O_ERR_ARG, "q, k, v, out must be non-NULL");
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t qb = (size_t)c->B * c->Hq * T * c->d * c->elem;
+    const size_t kb = (size_t)c->B * c->Hkv * T * c->d * c->elem;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t need = up(qb) * 2 + up(kb) * 2;  // q, out, k, v
+    if (!c->s_in) {
+        H2O_TRY(c, cudaStreamCreateWithFlags(&c->s_in, cudaStreamNonBlocking), "create upload stream");
+        H2O_TRY(c, cudaStreamCreateWithFlags(&c->s_out, cudaStreamNonBlocking), "create download stream");
+        for (int i = 0; i < 2; ++i)
+            for (cudaEvent_t* e : {&c->ev_in[i], &c->ev_step[i], &c->ev_out[i]})
+                H2O_TRY(c, cudaEventCreateWithFlags(e, cudaEventDisableTiming), "create pipeline event");
+    }
+    if (need > c->aslot_bytes) {  // grow both slots once every queued copy is done
+        H2O_TRY(c, cudaStreamSynchronize(c->s_in), "sync before staging growth");
+        H2O_TRY(c, cudaStreamSynchronize(c->s_out), "sync before staging growth");
+        H2O_TRY(c, cudaStreamSynchronize(s), "sync before staging growth");
+        for (int i = 0; i < 2; ++i) {
+            cudaFree(c->aslot[i]);
+            c->aslot[i] = nullptr;
+        }
+        c->aslot_bytes = 0;
+        for (int i = 0; i < 2; ++i) H2O_TRY(c, cudaMalloc(&c->aslot[i], need), "cudaMalloc(async staging)");
+        c->aslot_bytes = need;
+    }
+    const int sl = (int)(c->achunks & 1);
+    char* base = (char*)c->aslot[sl];
+    void* dq = base;
+    void* dout = base + up(qb);
+    void* dk = base + 2 * up(qb);
+    void* dv = base + 2 * up(qb) + up(kb);
+    // upload, once the step two chunks back has finished reading this slot
+    H2O_TRY(c, cudaStreamWaitEvent(c->s_in, c->ev_step[sl], 0), "order upload");
+    H2O_TRY(c, cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, c->s_in), "copy q to device");
+    H2O_TRY(c, cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, c->s_in), "copy k to device");
+    H2O_TRY(c, cudaMemcpyAsync(dv, v, kb, cudaMemcpyHostToDevice, c->s_in), "copy v to device");
+    H2O_TRY(c, cudaEventRecord(c->ev_in[sl], c->s_in), "record upload");
+    // the step, once the inputs are there and the slot's last output is downloaded
+    H2O_TRY(c, cudaStreamWaitEvent(s, c->ev_in[sl], 0), "order step");
+    H2O_TRY(c, cudaStreamWaitEvent(s, c->ev_out[sl], 0), "order step");
+    rc = h2o_step(c, dq, dk, dv, dout, T, stream);
+    if (rc != H2O_OK) return rc;
+    H2O_TRY(c, cudaEventRecord(c->ev_step[sl], s), "record step");
+    // download
+    H2O_TRY(c, cudaStreamWaitEvent(c->s_out, c->ev_step[sl], 0), "order download");
+    H2O_TRY(c, cudaMemcpyAsync(out, dout, qb, cudaMemcpyDeviceToHost, c->s_out), "copy out to host");
+    H2O_TRY(c, cudaEventRecord(c->ev_out[sl], c->s_out), "record download");
+    ++c->achunks;
+    return H2O_OK;
+}
+
+int h2o_host_sync(h2o_ctx* c) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    DeviceGuard g(c->device);
+    if (c->s_in) {
+        H2O_TRY(c, cudaStreamSynchronize(c->s_in), "synchronise uploads");
+        H2O_TRY(c, cudaStreamSynchronize(c->s_out), "synchronise downloads");
+    }
     return check_ctx(c);
 }
 

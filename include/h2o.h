@@ -100,6 +100,28 @@ int h2o_step(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *ou
 int h2o_step_host(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
                   int T, void *stream);
 
+/* Pipelined form of h2o_step_host for a run of chunks: enqueues the upload of
+ * (q, k, v) from HOST memory into one of two library-owned device staging
+ * slots (on an internal upload stream), the step (on `stream`) and the
+ * download of the output into out (HOST, on an internal download stream), and
+ * returns without waiting. Successive calls alternate the slots, so the
+ * upload of chunk c+1 and the download of chunk c-1 overlap the step of chunk
+ * c; events order each slot's reuse. Use page-locked host memory: pageable
+ * memory is correct but serialises the copies. q, k, v must stay unchanged
+ * and out must not be read until h2o_host_sync returns; chunks must be
+ * submitted in sequence order on one stream, and the other calls that touch
+ * the context (h2o_reset, h2o_get_state, ...) only after h2o_host_sync.
+ * Same shapes and errors as h2o_step; the first call creates the two streams
+ * and three events per slot, and a larger T than before grows both slots once
+ * (synchronising). The paper has no counterpart of this host interface. */
+int h2o_step_host_async(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
+                        int T, void *stream);
+
+/* Waits until every upload and download enqueued by h2o_step_host_async has
+ * finished (the outputs are in host memory), then reports any device error
+ * as h2o_sync_check does. The caller's `stream` is not synchronised. */
+int h2o_host_sync(h2o_ctx *ctx);
+
 /* Current H2O scores, float [B, Hkv, C] (device dst); 0 in empty slots. */
 int h2o_scores(h2o_ctx *ctx, float *dst, void *stream);
 

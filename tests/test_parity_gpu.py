@@ -125,6 +125,36 @@ def test_step_host_matches_device_step():
     assert torch.equal(a.scores(), b.scores())
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_step_host_async_matches_device_step(dtype):
+    """The pipelined host path (two staging slots, upload/download streams)
+    gives exactly the device path's outputs, scores and positions, with all
+    chunks enqueued before one host_sync; a longer chunk in the middle grows
+    the staging slots."""
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    d = 128 if dtype == "bf16" else 64
+    wl = synth.Workload("host-async", dtype, B=2, Hq=8, Hkv=2, d=d, C=256, T=96, N=96 * 6, seed=11,
+                        recipe="heavy", hh_frac=0.03)
+    a = H2OCache(2, 8, 2, d, 256, tdt, max_T=160)
+    b = H2OCache(2, 8, 2, d, 256, tdt, max_T=160)
+    lens = [96, 96, 160, 96, 33, 96]  # chunk lengths: growth, then shorter chunks
+    ins, outs_a, outs_b = [], [], []
+    for c, T in enumerate(lens):
+        q, k, v = (x[:, :, :T].copy() for x in synth.chunk(wl.with_(T=max(lens)), c))
+        qd, kd, vd = to_dev(q, dtype), to_dev(k, dtype), to_dev(v, dtype)
+        outs_a.append(a.step(qd, kd, vd).cpu())
+        host = tuple(t.cpu().pin_memory() for t in (qd, kd, vd))
+        ins.append(host)  # kept alive until host_sync
+        outs_b.append(torch.empty_like(host[0]).pin_memory())
+        b.step_host_async(*host, outs_b[-1])
+    b.host_sync()
+    torch.cuda.synchronize()
+    for oa, ob in zip(outs_a, outs_b):
+        assert torch.equal(oa, ob)
+    assert torch.equal(a.positions(), b.positions())
+    assert torch.equal(a.scores(), b.scores())
+
+
 def test_bounded_wait_reports_timeout():
     """A kernel waiting on a barrier nobody completes gives up and reports
     H2O_ERR_TIMEOUT; the CUDA context stays usable."""
