@@ -24,8 +24,12 @@ class BruteH2O:
     cache[b][g] maps position -> [key (d,), value (d,), score].
     """
 
-    def __init__(self, B: int, Hq: int, Hkv: int, d: int, C: int):
+    def __init__(self, B: int, Hq: int, Hkv: int, d: int, C: int, normalized: bool = False):
+        """normalized: rank eviction candidates by score / age (age = token
+        count after the step minus the position, the same section's improved
+        score) instead of by the score."""
         self.B, self.Hq, self.Hkv, self.d, self.C = B, Hq, Hkv, d, C
+        self.normalized = normalized
         self.G = Hq // Hkv
         self.P = 0
         self.cache = [[dict() for _ in range(Hkv)] for _ in range(B)]
@@ -67,7 +71,9 @@ class BruteH2O:
                 for idx, p in enumerate(positions):
                     cand[p][2] = cand[p][2] + add[idx]
                 scores[b].append({p: cand[p][2] for p in positions})
-                order = sorted(positions, key=lambda p: (cand[p][2], p), reverse=True)
+                t_now = self.P + T
+                rank = (lambda p: cand[p][2] / (t_now - p)) if self.normalized else (lambda p: cand[p][2])
+                order = sorted(positions, key=lambda p: (rank(p), p), reverse=True)
                 keep = set(order[: self.C])
                 kept_sets[b].append(keep)
                 self.cache[b][g] = {p: cand[p] for p in keep}

@@ -25,6 +25,13 @@
  *   - kept cache entries stay in their slots; the kept chunk tokens, in
  *     ascending position, fill the free slots (empty or evicted) in ascending
  *     slot order.
+ * Eviction policies (the ranking key; the stored score is phi in both):
+ *   - sum (policy 0): phi itself;
+ *   - normalized (policy 1), the same section's improved score: phi divided
+ *     by the candidate's age, (t - t_j)^-1 * phi, read with t = P + T the
+ *     token count after the step and t_j the candidate's position, so every
+ *     age is at least 1 (the page's superscript is garbled; this is the
+ *     plainest reading).
  *
  * Everything is fp64, plain loops, exp()/log() from libm. OpenMP only splits
  * independent (batch, KV head) groups or independent query rows; no result
@@ -129,7 +136,7 @@ static double logit(const double *qrow, const double *krow, int d, double scale)
  *                        chunk tokens); *n_cand receives their count
  *   token_slot [T]       where each chunk token went, -1 if dropped
  */
-static int group_step(int G, int d, int C, int T, int64_t P,
+static int group_step(int G, int d, int C, int T, int64_t P, int policy,
                       double *Kc, double *Vc, double *phi, int64_t *pos,
                       const double *q, const double *k, const double *v,
                       double *out, double *lse,
@@ -158,8 +165,9 @@ static int group_step(int G, int d, int C, int T, int64_t P,
     const double **vrow = (const double **)malloc(sizeof(double *) * (size_t)(n_cand > 0 ? n_cand : 1));
     double *delta = (double *)calloc((size_t)(n_cand > 0 ? n_cand : 1), sizeof(double));
     double *w = (double *)malloc(sizeof(double) * (size_t)(n_cand > 0 ? n_cand : 1));
-    if (!krow || !vrow || !delta || !w) {
-        free(krow); free(vrow); free(delta); free(w);
+    double *rank_key = (double *)malloc(sizeof(double) * (size_t)(n_cand > 0 ? n_cand : 1));
+    if (!krow || !vrow || !delta || !w || !rank_key) {
+        free(krow); free(vrow); free(delta); free(w); free(rank_key);
         return ORACLE_ERR_OOM;
     }
     for (int c = 0; c < n_valid; ++c) {
@@ -203,8 +211,11 @@ static int group_step(int G, int d, int C, int T, int64_t P,
     /* Step 3: updated scores (old score plus this step's weight sum). */
     for (int c = 0; c < n_cand; ++c) cand_score[c] += delta[c];
 
-    /* Steps 4 and 5: eviction and slot placement. */
-    int rc = h2o_oracle_select_group(C, T, n_cand, cand_score, cand_pos, cand_slot,
+    /* Steps 4 and 5: eviction (ranked by the policy's key) and slot placement. */
+    const int64_t t_after = P + T;
+    for (int c = 0; c < n_cand; ++c)
+        rank_key[c] = policy == 1 ? cand_score[c] / (double)(t_after - cand_pos[c]) : cand_score[c];
+    int rc = h2o_oracle_select_group(C, T, n_cand, rank_key, cand_pos, cand_slot,
                                      cand_kept, token_slot);
     if (rc == ORACLE_OK) {
         for (int c = 0; c < n_valid; ++c) {
@@ -225,7 +236,7 @@ static int group_step(int G, int d, int C, int T, int64_t P,
             pos[j] = P + t;
         }
     }
-    free(krow); free(vrow); free(delta); free(w);
+    free(krow); free(vrow); free(delta); free(w); free(rank_key);
     return rc;
 }
 
@@ -236,15 +247,16 @@ static int group_step(int G, int d, int C, int T, int64_t P,
  *   n_cand [B,Hkv]  token_slot [B,Hkv,T]
  * Query head h belongs to KV head h / (Hq/Hkv). Groups run in parallel.
  */
-int h2o_oracle_step(int B, int Hq, int Hkv, int d, int C, int T, int64_t P,
-                    double *Kc, double *Vc, double *phi, int64_t *pos,
-                    const double *q, const double *k, const double *v,
-                    double *out, double *lse,
-                    double *cand_score, int64_t *cand_pos, int32_t *cand_slot,
-                    uint8_t *cand_kept, int32_t *n_cand, int32_t *token_slot,
-                    int nthreads)
+int h2o_oracle_step_policy(int B, int Hq, int Hkv, int d, int C, int T, int64_t P, int policy,
+                           double *Kc, double *Vc, double *phi, int64_t *pos,
+                           const double *q, const double *k, const double *v,
+                           double *out, double *lse,
+                           double *cand_score, int64_t *cand_pos, int32_t *cand_slot,
+                           uint8_t *cand_kept, int32_t *n_cand, int32_t *token_slot,
+                           int nthreads)
 {
-    if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0 || d <= 0 || C <= 0 || T <= 0 || P < 0)
+    if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0 || d <= 0 || C <= 0 || T <= 0 || P < 0 ||
+        (policy != 0 && policy != 1))
         return ORACLE_ERR_ARG;
     const int G = Hq / Hkv;
     const int groups = B * Hkv;
@@ -259,7 +271,7 @@ int h2o_oracle_step(int B, int Hq, int Hkv, int d, int C, int T, int64_t P,
         const size_t cs = (size_t)bg * C;
         const size_t ct = (size_t)bg * (C + T);
         const size_t qo = ((size_t)b * Hq + (size_t)g * G) * T;
-        int rc = group_step(G, d, C, T, P,
+        int rc = group_step(G, d, C, T, P, policy,
                             Kc + cs * d, Vc + cs * d, phi + cs, pos + cs,
                             q + qo * d, k + (size_t)bg * T * d, v + (size_t)bg * T * d,
                             out + qo * d, lse + qo,
@@ -273,6 +285,20 @@ int h2o_oracle_step(int B, int Hq, int Hkv, int d, int C, int T, int64_t P,
         }
     }
     return rc_all;
+}
+
+/* The step under the sum policy (policy 0). */
+int h2o_oracle_step(int B, int Hq, int Hkv, int d, int C, int T, int64_t P,
+                    double *Kc, double *Vc, double *phi, int64_t *pos,
+                    const double *q, const double *k, const double *v,
+                    double *out, double *lse,
+                    double *cand_score, int64_t *cand_pos, int32_t *cand_slot,
+                    uint8_t *cand_kept, int32_t *n_cand, int32_t *token_slot,
+                    int nthreads)
+{
+    return h2o_oracle_step_policy(B, Hq, Hkv, d, C, T, P, 0, Kc, Vc, phi, pos, q, k, v, out, lse,
+                                  cand_score, cand_pos, cand_slot, cand_kept, n_cand, token_slot,
+                                  nthreads);
 }
 
 /*

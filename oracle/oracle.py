@@ -45,6 +45,8 @@ def lib():
         I = ctypes.c_int
         L.h2o_oracle_step.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 15 + [I]
         L.h2o_oracle_step.restype = I
+        L.h2o_oracle_step_policy.argtypes = [I, I, I, I, I, I, ctypes.c_int64, I] + [P] * 15 + [I]
+        L.h2o_oracle_step_policy.restype = I
         L.h2o_oracle_select_group.argtypes = [I, I, I, P, P, P, P, P]
         L.h2o_oracle_select_group.restype = I
         L.h2o_oracle_rows.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 6 + [I, P, P, P, I]
@@ -97,8 +99,15 @@ class StepResult:
     extra: dict = field(default_factory=dict)
 
 
-def step(state: State, q: np.ndarray, k: np.ndarray, v: np.ndarray, nthreads: int = 0) -> StepResult:
-    """One H2O step; mutates ``state`` in place and returns the step's outputs."""
+POLICY_SUM = 0         # rank candidates by the H2O score
+POLICY_NORMALIZED = 1  # rank by the score over the candidate's age, t = P + T
+
+
+def step(state: State, q: np.ndarray, k: np.ndarray, v: np.ndarray, nthreads: int = 0,
+         policy: int = POLICY_SUM) -> StepResult:
+    """One H2O step; mutates ``state`` in place and returns the step's outputs.
+    ``policy`` picks the eviction ranking key (the stored scores are the sums
+    under both)."""
     q = np.ascontiguousarray(q, np.float64)
     k = np.ascontiguousarray(k, np.float64)
     v = np.ascontiguousarray(v, np.float64)
@@ -113,7 +122,7 @@ def step(state: State, q: np.ndarray, k: np.ndarray, v: np.ndarray, nthreads: in
     ck = np.zeros((B, Hkv, C + T), np.uint8)
     nc = np.zeros((B, Hkv), np.int32)
     ts = np.full((B, Hkv, T), -1, np.int32)
-    rc = lib().h2o_oracle_step(B, Hq, Hkv, d, C, T, int(state.P),
+    rc = lib().h2o_oracle_step_policy(B, Hq, Hkv, d, C, T, int(state.P), int(policy),
                                _p(state.K), _p(state.V), _p(state.phi), _p(state.pos),
                                _p(q), _p(k), _p(v), _p(out), _p(lse),
                                _p(cs), _p(cp), _p(cslot), _p(ck), _p(nc), _p(ts), int(nthreads))

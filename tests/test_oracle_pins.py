@@ -27,15 +27,16 @@ def _val(s):
     return float(Fraction(s))
 
 
-def run_both(B, Hq, Hkv, d, C, T, n_chunks, gen):
+def run_both(B, Hq, Hkv, d, C, T, n_chunks, gen, normalized=False):
     """Run the oracle and the brute-force simulation over the same chunks and
     yield per-step results of both."""
     st = oracle.State.empty(B, Hkv, C, d)
-    br = brute.BruteH2O(B, Hq, Hkv, d, C)
+    br = brute.BruteH2O(B, Hq, Hkv, d, C, normalized=normalized)
+    policy = oracle.POLICY_NORMALIZED if normalized else oracle.POLICY_SUM
     for c in range(n_chunks):
         q, k, v = gen(c)
         n_before = st.n_valid.copy()
-        res = oracle.step(st, q, k, v)
+        res = oracle.step(st, q, k, v, policy=policy)
         bo, bl, bs, bk = br.step(q, k, v)
         yield c, n_before, st, res, (bo, bl, bs, bk)
 
@@ -51,8 +52,10 @@ def iid_gen(B, Hq, Hkv, d, T, seed, kscale=1.0):
 
 
 # ---------------------------------------------------------------- golden ---
-def test_hand_worked_example(oracle_lib):
-    g = json.load(open(os.path.join(GOLDEN, "worked_example_c2_t2.json")))
+@pytest.mark.parametrize("fname", ["worked_example_c2_t2.json", "worked_example_c2_t2_normalized.json"])
+def test_hand_worked_example(oracle_lib, fname):
+    g = json.load(open(os.path.join(GOLDEN, fname)))
+    policy = oracle.POLICY_NORMALIZED if g.get("policy") == "normalized" else oracle.POLICY_SUM
     s = g["shape"]
     st = oracle.State.empty(s["B"], s["Hkv"], s["C"], s["d"])
     T = s["T"]
@@ -60,7 +63,7 @@ def test_hand_worked_example(oracle_lib):
         q = np.array([_val(x) for x in ch["q"]]).reshape(1, 1, T, 1)
         k = np.array([_val(x) for x in ch["k"]]).reshape(1, 1, T, 1)
         v = np.array([_val(x) for x in ch["v"]]).reshape(1, 1, T, 1)
-        r = oracle.step(st, q, k, v)
+        r = oracle.step(st, q, k, v, policy=policy)
         n = int(r.n_cand[0, 0])
         np.testing.assert_allclose(r.out.ravel(), [_val(x) for x in ch["out"]], rtol=0, atol=1e-13)
         np.testing.assert_allclose(r.lse.ravel(), [_val(x) for x in ch["lse"]], rtol=0, atol=1e-13)
@@ -80,9 +83,11 @@ def test_hand_worked_example(oracle_lib):
     (1, 3, 3, 4, 3, 5, 3, 1.5),     # chunk longer than the cache (MHA)
     (1, 4, 1, 6, 7, 4, 4, 0.5),     # G = 4
 ])
-def test_oracle_matches_brute_force(oracle_lib, B, Hq, Hkv, d, C, T, n_chunks, kscale):
+@pytest.mark.parametrize("normalized", [False, True])
+def test_oracle_matches_brute_force(oracle_lib, B, Hq, Hkv, d, C, T, n_chunks, kscale, normalized):
     gen = iid_gen(B, Hq, Hkv, d, T, seed=C * 100 + T, kscale=kscale)
-    for c, n_before, st, res, (bo, bl, bs, bk) in run_both(B, Hq, Hkv, d, C, T, n_chunks, gen):
+    for c, n_before, st, res, (bo, bl, bs, bk) in run_both(B, Hq, Hkv, d, C, T, n_chunks, gen,
+                                                           normalized=normalized):
         np.testing.assert_allclose(res.out, bo, rtol=0, atol=1e-12)
         np.testing.assert_allclose(res.lse, bl, rtol=0, atol=1e-12)
         for b in range(B):
