@@ -224,6 +224,9 @@ def run_ours(args, rank, world, local_rank):
         f"in {time.time() - t0:.1f}s")
     out = torch.empty_like(chunks[0][0])
     cache = H2OCache(wl.B, wl.Hq, wl.Hkv, wl.d, wl.C, tdt, max_T=wl.T)
+    if args.policy == "normalized":
+        from h2o_kv_cache_step_b200._lib import H2O_POLICY_NORMALIZED
+        cache.set_policy(H2O_POLICY_NORMALIZED)
     plan = cache.kernel_plan(wl.T)
     stream = torch.cuda.current_stream()
 
@@ -381,6 +384,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
                    "C": wl.C, "T": wl.T, "N": wl.N, "chunks_per_step": wl.n_chunks,
                    "global_batch": wl.B * world, "seq_len": wl.N, "parallelism": f"replicas{world}",
+                   "policy": args.policy,
                    "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB resident per rank)"},
         "gpu_launches": sum(cnt for (_, cnt) in prof.values()),
         "kernel_plan": plan,
@@ -483,6 +487,8 @@ def main():
     ap.add_argument("--mode", default="prefill", choices=["prefill", "chunk"],
                     help="prefill: a bench step is a whole-sequence prefill (default); chunk: one "
                          "steady-state chunk step (for profiler captures)")
+    ap.add_argument("--policy", default="sum", choices=["sum", "normalized"],
+                    help="eviction ranking: the H2O score (default) or score / age")
     ap.add_argument("--cpu-groups", type=int, default=0,
                     help="KV groups in the oracle sample (default: host cores)")
     args = ap.parse_args()

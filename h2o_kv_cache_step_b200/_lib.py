@@ -21,6 +21,8 @@ H2O_ERR_CUDA = -4
 H2O_ERR_TIMEOUT = -5
 H2O_ERR_POISONED = -6
 H2O_ERR_UNSUPPORTED = -7
+H2O_POLICY_SUM = 0
+H2O_POLICY_NORMALIZED = 1
 H2O_BF16 = 0
 H2O_FP32 = 1
 
@@ -40,6 +42,7 @@ SIGNATURES = [
     ("h2o_step_host", _I, [_P, _P, _P, _P, _P, _I, _P]),
     ("h2o_step_host_async", _I, [_P, _P, _P, _P, _P, _I, _P]),
     ("h2o_host_sync", _I, [_P]),
+    ("h2o_set_policy", _I, [_P, _I]),
     ("h2o_scores", _I, [_P, _P, _P]),
     ("h2o_positions", _I, [_P, _P, _P]),
     ("h2o_counters", _I, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),

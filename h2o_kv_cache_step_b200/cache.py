@@ -76,6 +76,11 @@ class H2OCache:
                                    _stream_ptr(stream)))
         return out
 
+    def set_policy(self, policy: int) -> None:
+        """Eviction ranking for the following steps: _lib.H2O_POLICY_SUM (the
+        H2O score, default) or _lib.H2O_POLICY_NORMALIZED (score / age)."""
+        self._check(lib().h2o_set_policy(self._h, int(policy)))
+
     def _check_host(self, q, k, v, out) -> int:
         T = q.shape[2]
         for name, t, heads in (("q", q, self.Hq), ("k", k, self.Hkv), ("v", v, self.Hkv), ("out", out, self.Hq)):

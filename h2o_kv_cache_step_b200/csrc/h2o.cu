@@ -38,6 +38,7 @@ void h2o::set_thread_error_message(const char* msg) {
 
 struct h2o_ctx {
     int B, Hq, Hkv, d, C, dtype, tmax;
+    int policy = 0;  // H2O_POLICY_SUM
     int device;
     int num_sms;
     int64_t P, n;
@@ -203,6 +204,7 @@ StepArgs make_args(h2o_ctx* c, const void* q, const void* k, const void* v, void
     a.n = (int)c->n;
     a.P = c->P;
     a.dtype = c->dtype;
+    a.policy = c->policy;
     a.tmax = c->tmax;
     a.q = q;
     a.k = k;
@@ -485,6 +487,14 @@ int h2o_step_host_async(h2o_ctx* c, const void* q, const void* k, const void* v,
     H2O_TRY(c, cudaMemcpyAsync(out, dout, qb, cudaMemcpyDeviceToHost, c->s_out), "copy out to host");
     H2O_TRY(c, cudaEventRecord(c->ev_out[sl], c->s_out), "record download");
     ++c->achunks;
+    return H2O_OK;
+}
+
+int h2o_set_policy(h2o_ctx* c, int policy) {
+    if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
+    if (policy != H2O_POLICY_SUM && policy != H2O_POLICY_NORMALIZED)
+        return fail(c, H2O_ERR_ARG, "unknown eviction policy %d", policy);
+    c->policy = policy;
     return H2O_OK;
 }
 

@@ -28,6 +28,7 @@ struct StepArgs {
     int n;            // valid cache slots (prefix 0..n-1) before the step
     int64_t P;        // position of the chunk's first token
     int dtype;        // 0 = bf16, 1 = fp32
+    int policy;       // eviction ranking: 0 = H2O score, 1 = score / age
     int tmax;         // capacity (in tokens) of the per-step workspace
     const void* q;    // [B,Hq,T,d]
     const void* k;    // [B,Hkv,T,d]

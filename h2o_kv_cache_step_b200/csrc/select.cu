@@ -30,8 +30,18 @@ __device__ __forceinline__ uint32_t ordered_bits(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ uint64_t cand_key(const float* cs, const int32_t* cp, int c) {
-    return ((uint64_t)ordered_bits(cs[c]) << 32) | (uint32_t)cp[c];
+// Eviction ranking value of a candidate: its H2O score (sum policy), or the
+// score over its age t - t_j with t = P + T the token count after the step
+// (normalized policy; "Learning how to Forget", paper page, section
+// "Improvements to Heavy-Hitter Oracle (H2O)"). fp32, division rounded to
+// nearest, so that a host replay in fp32 ranks identically.
+__device__ __forceinline__ float rank_value(float score, int32_t pos, int policy, long long t_after) {
+    return policy == 1 ? __fdiv_rn(score, (float)(t_after - (long long)pos)) : score;
+}
+
+__device__ __forceinline__ uint64_t cand_key(const float* cs, const int32_t* cp, int c, int policy,
+                                             long long t_after) {
+    return ((uint64_t)ordered_bits(rank_value(cs[c], cp[c], policy, t_after)) << 32) | (uint32_t)cp[c];
 }
 
 // Candidate keys are staged in shared memory when they fit (the radix passes
@@ -80,7 +90,8 @@ __global__ void __launch_bounds__(kSelThreads)
 select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
               uint8_t* __restrict__ cand_kept, int32_t* __restrict__ token_slot,
               int32_t* __restrict__ free_list, float* __restrict__ scores, int32_t* __restrict__ pos,
-              const float* __restrict__ partials, int nparts, int C, int T, int n, int tmax, long long P) {
+              const float* __restrict__ partials, int nparts, int C, int T, int n, int tmax, long long P,
+              int policy) {
     __shared__ unsigned int hist[256];
     __shared__ unsigned long long scan_scratch[33];
     __shared__ unsigned long long red_min[32], red_max[32];
@@ -152,7 +163,8 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
                 cs[c] = sv[u];
                 cp[c] = pv[u];
             }
-            const unsigned long long key = ((uint64_t)ordered_bits(sv[u]) << 32) | (uint32_t)pv[u];
+            const unsigned long long key =
+                ((uint64_t)ordered_bits(rank_value(sv[u], pv[u], policy, P + T)) << 32) | (uint32_t)pv[u];
             if (SMEM_KEYS) skeys[c] = key;
             kmin = key < kmin ? key : kmin;
             kmax = key > kmax ? key : kmax;
@@ -191,7 +203,9 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         sh_done = (m <= C) || sh_hi == 0;
     }
     __syncthreads();
-    auto key_of = [&](int c) -> uint64_t { return SMEM_KEYS ? (uint64_t)skeys[c] : cand_key(cs, cp, c); };
+    auto key_of = [&](int c) -> uint64_t {
+        return SMEM_KEYS ? (uint64_t)skeys[c] : cand_key(cs, cp, c, policy, P + T);
+    };
 
     // ---- 1. threshold: the C-th largest key, MSB-first radix select over the
     // bits below the shared prefix, 8 bits a pass; it stops as soon as the
@@ -353,11 +367,11 @@ cudaError_t launch_select(const StepArgs& a) {
     if (with_keys <= (size_t)kSelectSmemLimit) {
         e = launch_ex(kEarlyLaunch, select_kernel<true>, dim3(a.B * a.Hkv), dim3(kSelThreads), with_keys, a.stream, a.cand_score,
                        a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
-                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
+                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P, a.policy);
     } else if (tail <= (size_t)kSelectSmemLimit) {
         e = launch_ex(kEarlyLaunch, select_kernel<false>, dim3(a.B * a.Hkv), dim3(kSelThreads), tail, a.stream, a.cand_score,
                        a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
-                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P);
+                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P, a.policy);
     } else {
         return cudaErrorInvalidConfiguration;
     }

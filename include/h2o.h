@@ -73,6 +73,16 @@ enum h2o_status {
 
 enum h2o_dtype { H2O_BF16 = 0, H2O_FP32 = 1 };
 
+/* Eviction ranking ("Learning how to Forget", paper page, section
+ * "Improvements to Heavy-Hitter Oracle (H2O)"): candidates are ranked by
+ *   H2O_POLICY_SUM         their H2O score phi (the default), or
+ *   H2O_POLICY_NORMALIZED  phi / (t - t_j): the score over the candidate's age,
+ *                          with t = P + T the token count after the step and
+ *                          t_j the candidate's position (every age >= 1).
+ * Ties go to the larger position under both. The stored scores are phi
+ * under both policies; only the ranking key differs. */
+enum h2o_policy { H2O_POLICY_SUM = 0, H2O_POLICY_NORMALIZED = 1 };
+
 /* Create a bf16 context on the current CUDA device: an empty cache of C slots
  * per (sequence, KV head), P = 0. Allocates all device memory it will need for
  * chunks of up to T = C tokens (larger chunks grow the workspace once).
@@ -90,6 +100,10 @@ int h2o_destroy(h2o_ctx *ctx);
 /* One H2O step on the chunk (q, k, v) of T tokens (device pointers, layouts
  * above); writes the attention output to out (device). Updates the cache,
  * scores and positions; P advances by T. Asynchronous on `stream`. */
+/* Select the eviction ranking (enum h2o_policy) for the following steps.
+ * Takes effect from the next h2o_step; H2O_ERR_ARG for an unknown policy. */
+int h2o_set_policy(h2o_ctx *ctx, int policy);
+
 int h2o_step(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
              int T, void *stream);
 
@@ -204,7 +218,8 @@ int h2o_profile_end(h2o_ctx *ctx, int max_kernels, const char **names, double *t
  * Given, for `groups` (sequence, KV head) groups, the updated candidate scores
  * and positions of one step (device float / int32 [groups, n+T]: cache slots
  * 0..n-1, then the T chunk tokens at positions P..P+T-1), it computes what
- * h2o_step's eviction computes: kept flags (device uint8 [groups, n+T]), the
+ * h2o_step's eviction computes under H2O_POLICY_SUM (it ranks by the scores
+ * as given): kept flags (device uint8 [groups, n+T]), the
  * slot of each chunk token or -1 (device int32 [groups, T]), and updates the
  * slot scores and positions (device float / int32 [groups, C], in/out: kept
  * cache slots take their new score, kept chunk tokens fill the free slots in

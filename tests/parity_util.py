@@ -56,14 +56,26 @@ def gpu_step(cache, q, k, v, dtype):
     return r
 
 
-def check_selection_replay(g, pre: oracle.State, k, v, C, T):
+def ranking_keys(cand_score, cand_pos, t_after, policy):
+    """The eviction ranking key the device uses, in the device's precision:
+    the fp32 score, or (normalized policy) the fp32 score divided by the fp32
+    age t_after - pos, rounded to nearest. Returned as float64 (exact)."""
+    s = np.asarray(cand_score, np.float32)
+    if policy == oracle.POLICY_NORMALIZED:
+        age = (np.int64(t_after) - np.asarray(cand_pos, np.int64)).astype(np.float32)
+        s = (s / age).astype(np.float32)
+    return s.astype(np.float64)
+
+
+def check_selection_replay(g, pre: oracle.State, k, v, C, T, policy=oracle.POLICY_SUM):
     """Replay the oracle's selection on the GPU's candidate scores; kept flags,
     token slots and the new slot contents must match bit for bit."""
     B, Hkv = g["cand_score"].shape[:2]
     n_prev = g["cand_score"].shape[2] - T
+    t_after = int(pre.P) + T
     for b in range(B):
         for gg in range(Hkv):
-            cs = g["cand_score"][b, gg].astype(np.float64)
+            cs = ranking_keys(g["cand_score"][b, gg], g["cand_pos"][b, gg], t_after, policy)
             cp = g["cand_pos"][b, gg].astype(np.int64)
             slot = np.concatenate([np.arange(n_prev, dtype=np.int32), np.full(T, -1, np.int32)])
             kept, ts = oracle.select_group(C, T, cs, cp, slot)
@@ -100,11 +112,11 @@ def compare_scores(gpu_scores, ref_scores, what=""):
     return float((err / (np.abs(ref_scores) + SCORE_ATOL)).max())
 
 
-def lockstep_full(cache, q, k, v, dtype, C):
+def lockstep_full(cache, q, k, v, dtype, C, policy=oracle.POLICY_SUM):
     """One lockstep step with the full oracle step; returns stats."""
     pre = oracle_state_from_device(cache)
     ref_state = pre.copy()
-    res = oracle.step(ref_state, q, k, v)
+    res = oracle.step(ref_state, q, k, v, policy=policy)
     g = gpu_step(cache, q, k, v, dtype)
     T = q.shape[2]
     out_err = float(np.abs(g["out"] - res.out).max())
@@ -116,6 +128,6 @@ def lockstep_full(cache, q, k, v, dtype, C):
     assert (res.n_cand == nc).all()
     assert np.array_equal(g["cand_pos"], res.cand_pos[:, :, :nc].astype(np.int32))
     score_rel = compare_scores(g["cand_score"], res.cand_score[:, :, :nc], "candidate scores")
-    check_selection_replay(g, pre, k, v, C, T)
+    check_selection_replay(g, pre, k, v, C, T, policy)
     same_sel = bool(np.array_equal(g["kept"], res.cand_kept[:, :, :nc]))
     return dict(out_err=out_err, lse_err=lse_err, score_rel=score_rel, same_selection=same_sel)

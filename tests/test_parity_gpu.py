@@ -67,6 +67,40 @@ def test_short_chunks_lockstep(T):
         lockstep_full(cache, q, k, v, "bf16", wl.C)
 
 
+@pytest.mark.parametrize("dtype,d,B,Hq,Hkv,C,T,chunks", [
+    ("fp32", 64, 1, 4, 2, 256, 64, 8),       # the tiny workload's shape, 4 evicting steps
+    ("bf16", 128, 2, 8, 2, 384, 200, 4),     # ragged T and C, GQA 4
+    ("bf16", 64, 1, 8, 1, 300, 130, 4),      # d = 64, one KV head, G = 8
+    ("bf16", 128, 1, 4, 2, 100, 300, 3),     # chunk longer than the cache
+])
+def test_normalized_policy_lockstep(dtype, d, B, Hq, Hkv, C, T, chunks):
+    """Eviction ranked by score / age (H2O_POLICY_NORMALIZED): outputs and
+    scores against the oracle under the same policy, selection bit-exact on
+    replay with the device's fp32 key."""
+    from h2o_kv_cache_step_b200._lib import H2O_POLICY_NORMALIZED
+    wl = synth.Workload("norm", dtype, B=B, Hq=Hq, Hkv=Hkv, d=d, C=C, T=T, N=T * chunks,
+                        seed=13, recipe="heavy", hh_frac=0.05)
+    cache = H2OCache(wl.B, wl.Hq, wl.Hkv, wl.d, wl.C, TORCH_DTYPE[dtype], max_T=wl.T)
+    cache.set_policy(H2O_POLICY_NORMALIZED)
+    differs = False
+    for c in range(wl.n_chunks):
+        q, k, v = synth.chunk(wl, c)
+        pre = oracle_state_from_device(cache)
+        lockstep_full(cache, q, k, v, dtype, wl.C, policy=oracle.POLICY_NORMALIZED)
+        # the policy matters: the sum policy would keep another set somewhere
+        r_sum = oracle.step(pre.copy(), q, k, v, policy=oracle.POLICY_SUM)
+        r_norm = oracle.step(pre.copy(), q, k, v, policy=oracle.POLICY_NORMALIZED)
+        differs |= not np.array_equal(r_sum.cand_kept, r_norm.cand_kept)
+    assert differs
+
+
+def test_set_policy_rejects_unknown():
+    from h2o_kv_cache_step_b200._lib import H2OError
+    cache = H2OCache(1, 2, 1, 64, 8, torch.float32, max_T=4)
+    with pytest.raises(H2OError):
+        cache.set_policy(7)
+
+
 def test_cache_of_one_slot():
     wl = synth.Workload("c1slot", "fp32", B=1, Hq=2, Hkv=1, d=64, C=1, T=5, N=20, seed=2)
     run_sequence_lockstep(wl)
@@ -186,8 +220,9 @@ FULL = [w for w in synth.WORKLOAD_ORDER if w != "tiny-fp32"]
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(name):
+@pytest.mark.parametrize("name,policy", [(n, oracle.POLICY_SUM) for n in FULL] +
+                         [(FULL[0], oracle.POLICY_NORMALIZED)])
+def test_full_size_sampled(name, policy):
     """One steady-state step at the workload's full size: a full cache
     (random scores and scattered positions) and one real chunk. Checks
     sampled output rows and LSEs, every candidate score of one whole group,
@@ -195,6 +230,7 @@ def test_full_size_sampled(name):
     wl = synth.WORKLOADS[name]
     P = wl.C + 3 * wl.T  # a mid-sequence position
     cache = H2OCache(wl.B, wl.Hq, wl.Hkv, wl.d, wl.C, torch.bfloat16, max_T=wl.T)
+    cache.set_policy(policy)
     K, V, S, pos = synth.random_state(wl, n=wl.C, P=P, seed=99)
     cache.set_state(to_dev(K, "bf16"), to_dev(V, "bf16"), torch.from_numpy(S).cuda(),
                     torch.from_numpy(pos).cuda(), P=P, n=wl.C)
@@ -217,8 +253,8 @@ def test_full_size_sampled(name):
     sub = oracle.State(pre.K[b:b + 1, gg:gg + 1].copy(), pre.V[b:b + 1, gg:gg + 1].copy(),
                        pre.phi[b:b + 1, gg:gg + 1].copy(), pre.pos[b:b + 1, gg:gg + 1].copy(), pre.P)
     res = oracle.step(sub, q[b:b + 1, gg * G:(gg + 1) * G], k[b:b + 1, gg:gg + 1], v[b:b + 1, gg:gg + 1],
-                      nthreads=8)
+                      nthreads=8, policy=policy)
     nc = wl.C + T
     compare_scores(g["cand_score"][b, gg], res.cand_score[0, 0, :nc], f"{name} group scores")
     assert np.abs(g["out"][b, gg * G:(gg + 1) * G] - res.out[0]).max() <= TOL_OUT["bf16"]
-    check_selection_replay(g, pre, k, v, wl.C, T)
+    check_selection_replay(g, pre, k, v, wl.C, T, policy)
