@@ -248,6 +248,24 @@ def run_ours(args, rank, world, local_rank):
             cache.set_state(*st, P=c_idx * wl.T, n=wl.C)
             cache.step(*chunks[c_idx], out=out)
 
+    if args.mode == "decode":
+        # a bench step: a full cache (C slots, scattered positions), then
+        # `decode_steps` steps of `decode_t` new tokens each
+        dT, D = args.decode_t, args.decode_steps
+        dwl = wl.with_(T=dT, N=dT * D)
+        dchunks = [tuple(torch.from_numpy(x).to(dev).to(tdt) for x in synth.chunk(dwl, c)) for c in range(D)]
+        P0 = 2 * wl.C
+        K0, V0, S0, pos0 = synth.random_state(wl, n=wl.C, P=P0, seed=1)
+        st = tuple(torch.from_numpy(x).to(dev) for x in (K0, V0, S0, pos0))
+        st = (st[0].to(tdt), st[1].to(tdt), st[2], st[3])
+        sched = [(wl.C, dT)] * D
+        dout = torch.empty_like(dchunks[0][0])
+
+        def prefill():  # noqa: F811
+            cache.set_state(*st, P=P0, n=wl.C)
+            for (q, k, v) in dchunks:
+                cache.step(q, k, v, out=dout)
+
     for _ in range(args.warmup):
         prefill()
     cache.sync_check()
@@ -286,7 +304,8 @@ def run_ours(args, rank, world, local_rank):
 
     ms_total = max_over_ranks(ms_total, dev)
     ms_per_step = ms_total / args.steps
-    tokens_per_rank = (wl.B * wl.N if args.mode == "prefill" else wl.B * wl.T) * args.steps
+    tokens_per_rank = {"prefill": wl.B * wl.N, "chunk": wl.B * wl.T,
+                       "decode": wl.B * args.decode_t * args.decode_steps}[args.mode] * args.steps
     value = job_throughput(tokens_per_rank, world, ms_total)
 
     # roofline of the dominant kernel
@@ -384,7 +403,9 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
                    "C": wl.C, "T": wl.T, "N": wl.N, "chunks_per_step": wl.n_chunks,
                    "global_batch": wl.B * world, "seq_len": wl.N, "parallelism": f"replicas{world}",
-                   "policy": args.policy,
+                   "policy": args.policy, "mode": args.mode,
+                   **({"decode_t": args.decode_t, "decode_steps": args.decode_steps}
+                      if args.mode == "decode" else {}),
                    "l2": f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB resident per rank)"},
         "gpu_launches": sum(cnt for (_, cnt) in prof.values()),
         "kernel_plan": plan,
@@ -484,9 +505,12 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="prefill", choices=["prefill", "chunk"],
+    ap.add_argument("--decode-t", type=int, default=1, help="tokens per decode step (--mode decode)")
+    ap.add_argument("--decode-steps", type=int, default=256, help="decode steps per bench step")
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "chunk", "decode"],
                     help="prefill: a bench step is a whole-sequence prefill (default); chunk: one "
-                         "steady-state chunk step (for profiler captures)")
+                         "steady-state chunk step (for profiler captures); decode: --decode-steps "
+                         "steps of --decode-t tokens against a full cache")
     ap.add_argument("--policy", default="sum", choices=["sum", "normalized"],
                     help="eviction ranking: the H2O score (default) or score / age")
     ap.add_argument("--cpu-groups", type=int, default=0,

@@ -59,6 +59,10 @@ struct h2o_ctx {
     size_t partial_elems = 0;
     float* nlse2 = nullptr;
     int rows_pad = 0;
+    // decode-path workspace (chunks of up to kDecodeMaxT tokens)
+    float* dec_part = nullptr;
+    float* dec_logits = nullptr;
+    float* dec_lse2 = nullptr;
     // host staging for h2o_step_host
     void* stage = nullptr;
     size_t stage_bytes = 0;
@@ -156,6 +160,10 @@ void free_workspace(h2o_ctx* c) {
     cudaFree(c->token_slot);
     cudaFree(c->partials);
     cudaFree(c->nlse2);
+    cudaFree(c->dec_part);
+    cudaFree(c->dec_logits);
+    cudaFree(c->dec_lse2);
+    c->dec_part = c->dec_logits = c->dec_lse2 = nullptr;
     c->nlse2 = nullptr;
     c->lse = c->cand_score = c->partials = nullptr;
     c->cand_pos = c->token_slot = nullptr;
@@ -176,6 +184,14 @@ int alloc_workspace(h2o_ctx* c, int tmax) {
         H2O_TRY(c, cudaMalloc(&c->partials, sizeof(float) * c->partial_elems), "cudaMalloc(partials)");
     c->rows_pad = tc_rows_pad(c->Hq, c->Hkv, tmax);
     H2O_TRY(c, cudaMalloc(&c->nlse2, sizeof(float) * groups * (size_t)c->rows_pad), "cudaMalloc(nlse2)");
+    if (decode_applies(c->Hq, c->Hkv, c->d, 1)) {
+        H2O_TRY(c, cudaMalloc(&c->dec_part, sizeof(float) * decode_part_floats(c->B, c->Hq, c->Hkv, c->d, c->C)),
+                "cudaMalloc(decode partials)");
+        H2O_TRY(c, cudaMalloc(&c->dec_logits, sizeof(float) * decode_logit_floats(c->B, c->Hkv, c->C)),
+                "cudaMalloc(decode logits)");
+        H2O_TRY(c, cudaMalloc(&c->dec_lse2, sizeof(float) * decode_lse2_floats(c->B, c->Hkv)),
+                "cudaMalloc(decode lse)");
+    }
     c->tmax = tmax;
     return H2O_OK;
 }
@@ -223,6 +239,9 @@ StepArgs make_args(h2o_ctx* c, const void* q, const void* k, const void* v, void
     a.partials = c->partials;
     a.partial_elems = c->partial_elems;
     a.nlse2 = c->nlse2;
+    a.dec_part = c->dec_part;
+    a.dec_logits = c->dec_logits;
+    a.dec_lse2 = c->dec_lse2;
     a.rows_pad = c->rows_pad;
     a.wb.err_word = c->err_dev;
     a.wb.ns = c->wait_ns;
@@ -341,7 +360,11 @@ int h2o_kernel_plan(const h2o_ctx* c, int T, const char** names, int max_names) 
     if (!c || T < 1) return fail(nullptr, H2O_ERR_ARG, "bad arguments");
     const char* plan[kMaxStepKernels];
     int k = 0;
-    if (c->use_tc) {
+    if (c->dec_part && decode_applies(c->Hq, c->Hkv, c->d, T)) {
+        plan[k++] = "decode_split_kernel";
+        plan[k++] = "decode_combine_kernel";
+        plan[k++] = "decode_wsum_kernel";
+    } else if (c->use_tc) {
         k = tc_kernel_plan(c->B, c->Hq, c->Hkv, c->d, c->C, T, (int)c->n, plan, kMaxStepKernels - 2);
     } else {
         plan[k++] = "sdpa_simt_kernel";
@@ -381,8 +404,11 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
         a.log->ev = &c->prof_ev[(size_t)slot * (kMaxStepKernels + 1)];
         H2O_TRY(c, cudaEventRecord(a.log->ev[0], s), "record profiling event");
     }
-    a.nparts = c->use_tc ? tc_partial_count(c->Hq, c->Hkv, T) : 0;
-    if (c->use_tc) {
+    const bool decode = c->dec_part && decode_applies(c->Hq, c->Hkv, c->d, T);
+    a.nparts = decode ? 1 : c->use_tc ? tc_partial_count(c->Hq, c->Hkv, T) : 0;
+    if (decode) {
+        H2O_TRY(c, launch_decode(a), "launch decode-path kernels");
+    } else if (c->use_tc) {
         H2O_TRY(c, tc_sdpa(a), "launch tensor-core SDPA");
         H2O_TRY(c, tc_wsum(a), "launch tensor-core weight sums");
     } else {

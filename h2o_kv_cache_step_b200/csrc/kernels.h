@@ -49,6 +49,9 @@ struct StepArgs {
     float* partials;     // weight-sum partials [nparts][B*Hkv][C+tmax] (tensor-core path)
     size_t partial_elems;
     int nparts;          // > 0: the selection kernel first sums the partials
+    float* dec_part;     // decode path: per-(group, slice, row) partial O, max, sum
+    float* dec_logits;   // decode path: scaled logits [group][row][C + kDecodeMaxT]
+    float* dec_lse2;     // decode path: log2-sum-exp per (group, row)
     const void* tmaps;   // device copy of the step's TMA descriptors (tensor-core path)
     WaitBound wb;
     cudaStream_t stream;
@@ -93,6 +96,20 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 cudaError_t launch_sdpa_simt(const StepArgs& a);
 cudaError_t launch_wsum_simt(const StepArgs& a);
 // Eviction: per (sequence, KV head) radix select + slot map, then K/V copy.
+// Decode path (short chunks): split-K SDPA, combine, weight sums from the
+// kept logits; then launch_select with nparts = 1 and launch_scatter.
+constexpr int kDecodeMaxT = 16;      // longest chunk the decode path takes
+// query rows per KV group (G * T) it takes: the split kernel's dot products
+// run on the CUDA cores, and above this the tensor-core chunk path is faster
+// (measured: 64 rows, T = 16 at G = 4: 113 us per step here against 73)
+constexpr int kDecodeMaxRows = 32;
+constexpr int kDecodeSplit = 64;     // cache slots per split
+bool decode_applies(int Hq, int Hkv, int d, int T);
+size_t decode_part_floats(int B, int Hq, int Hkv, int d, int C);
+size_t decode_logit_floats(int B, int Hkv, int C);
+size_t decode_lse2_floats(int B, int Hkv);
+cudaError_t launch_decode(const StepArgs& a);
+
 cudaError_t launch_select(const StepArgs& a);
 cudaError_t launch_scatter(const StepArgs& a);
 // Sets the message h2o_last_error(NULL) reports on this thread.

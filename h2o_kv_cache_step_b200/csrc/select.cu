@@ -81,6 +81,7 @@ __device__ V block_exclusive_scan(V v, V* scratch, V* total) {
 }
 
 constexpr int kCandPerThread = 4;  // candidates a thread loads per round
+constexpr int kFewEvictions = 8;   // up to this many evictions: repeated block minima
 constexpr int kPartBatch = 4;      // weight-sum partials loaded per batch
 
 // One CTA per (sequence, KV head). Shared memory: the 64-bit candidate keys
@@ -95,7 +96,7 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     __shared__ unsigned int hist[256];
     __shared__ unsigned long long scan_scratch[33];
     __shared__ unsigned long long red_min[32], red_max[32];
-    __shared__ unsigned long long sh_prefix;
+    __shared__ unsigned long long sh_prefix, sh_prefix_min;
     __shared__ int sh_hi, sh_krem, sh_done;
     extern __shared__ __align__(16) unsigned char dyn[];
 
@@ -201,11 +202,49 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         sh_prefix = sh_hi >= 64 ? 0ull : (kmax >> sh_hi);
         sh_krem = C;
         sh_done = (m <= C) || sh_hi == 0;
+        sh_prefix_min = kmin;
     }
     __syncthreads();
     auto key_of = [&](int c) -> uint64_t {
         return SMEM_KEYS ? (uint64_t)skeys[c] : cand_key(cs, cp, c, policy, P + T);
     };
+
+    // few evictions (short chunks): the threshold is the k-th smallest key,
+    // found by k - 1 block minima above the smallest one; no radix pass
+    if (m > C && m - C <= kFewEvictions) {
+        unsigned long long thr = sh_prefix_min;
+        for (int it = 1; it < m - C; ++it) {
+            unsigned long long lm = ~0ull;
+            for (int c = threadIdx.x; c < m; c += blockDim.x) {
+                const unsigned long long key = key_of(c);
+                if (key > thr && key < lm) lm = key;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const unsigned long long o = __shfl_xor_sync(0xffffffffu, lm, off);
+                lm = o < lm ? o : lm;
+            }
+            if (lane == 0) red_min[warp] = lm;
+            __syncthreads();
+            if (warp == 0) {
+                lm = lane < (int)(blockDim.x >> 5) ? red_min[lane] : ~0ull;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const unsigned long long o = __shfl_xor_sync(0xffffffffu, lm, off);
+                    lm = o < lm ? o : lm;
+                }
+                if (lane == 0) sh_prefix_min = lm;
+            }
+            __syncthreads();
+            thr = sh_prefix_min;
+        }
+        if (threadIdx.x == 0) {  // kept iff key > thr
+            sh_hi = 0;
+            sh_prefix = thr + 1ull;
+            sh_done = 1;
+        }
+        __syncthreads();
+    }
 
     // ---- 1. threshold: the C-th largest key, MSB-first radix select over the
     // bits below the shared prefix, 8 bits a pass; it stops as soon as the

@@ -101,6 +101,45 @@ def test_set_policy_rejects_unknown():
         cache.set_policy(7)
 
 
+@pytest.mark.parametrize("dtype,d,Hq,Hkv,C,T,policy", [
+    ("bf16", 128, 8, 2, 300, 1, 0),    # one token per step: classic decode
+    ("bf16", 128, 32, 8, 256, 4, 0),   # the bench layer's heads, G = 4
+    ("bf16", 64, 8, 1, 200, 4, 0),     # G * T = 32 rows, the most the decode path takes
+    ("fp32", 128, 2, 2, 100, 16, 0),   # T = 16, the longest decode chunk (MHA)
+    ("fp32", 64, 4, 2, 130, 3, 0),
+    ("bf16", 128, 8, 2, 300, 2, 1),    # normalized policy
+])
+def test_decode_path_lockstep(dtype, d, Hq, Hkv, C, T, policy):
+    """Chunks of T <= 16 tokens take the split-K decode kernels; lockstep
+    against the oracle from a full cache with scattered positions, plus a
+    cold start (empty cache, a single split)."""
+    wl = synth.Workload("decode", dtype, B=2, Hq=Hq, Hkv=Hkv, d=d, C=C, T=T, N=T * 6, seed=21,
+                        recipe="heavy", hh_frac=0.05)
+    cache = H2OCache(wl.B, wl.Hq, wl.Hkv, wl.d, wl.C, TORCH_DTYPE[dtype], max_T=16)
+    assert cache.kernel_plan(T)[0] == "decode_split_kernel"
+    cache.set_policy(policy)
+    for c in range(2):  # cold start
+        q, k, v = synth.chunk(wl, c)
+        lockstep_full(cache, q, k, v, dtype, wl.C, policy=policy)
+    K, V, S, pos = synth.random_state(wl, n=wl.C, P=1000, seed=T)
+    cache.set_state(to_dev(K, dtype), to_dev(V, dtype), torch.from_numpy(S).cuda(),
+                    torch.from_numpy(pos).cuda(), P=1000, n=wl.C)
+    for c in range(2, wl.n_chunks):
+        q, k, v = synth.chunk(wl, c)
+        lockstep_full(cache, q, k, v, dtype, wl.C, policy=policy)
+
+
+def test_decode_path_limits():
+    """Chunks with more than 32 query rows per KV group, or T > 16, take the
+    chunk path."""
+    cache = H2OCache(1, 8, 2, 128, 256, torch.bfloat16, max_T=64)
+    assert cache.kernel_plan(8)[0] == "decode_split_kernel"      # 4 heads x 8 = 32 rows
+    assert cache.kernel_plan(16)[0] == "sdpa_tc_kernel"          # 64 rows
+    cache2 = H2OCache(1, 2, 2, 64, 64, torch.float32, max_T=64)
+    assert cache2.kernel_plan(16)[0] == "decode_split_kernel"
+    assert cache2.kernel_plan(17)[0] == "sdpa_simt_kernel"
+
+
 def test_cache_of_one_slot():
     wl = synth.Workload("c1slot", "fp32", B=1, Hq=2, Hkv=1, d=64, C=1, T=5, N=20, seed=2)
     run_sequence_lockstep(wl)
