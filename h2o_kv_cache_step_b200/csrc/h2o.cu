@@ -54,7 +54,6 @@ struct h2o_ctx {
     int32_t* cand_pos = nullptr;
     uint8_t* cand_kept = nullptr;
     int32_t* token_slot = nullptr;
-    int32_t* free_list = nullptr;
     float* partials = nullptr;
     size_t partial_elems = 0;
     float* nlse2 = nullptr;
@@ -235,7 +234,6 @@ StepArgs make_args(h2o_ctx* c, const void* q, const void* k, const void* v, void
     a.cand_pos = c->cand_pos;
     a.cand_kept = c->cand_kept;
     a.token_slot = c->token_slot;
-    a.free_list = c->free_list;
     a.partials = c->partials;
     a.partial_elems = c->partial_elems;
     a.nlse2 = c->nlse2;
@@ -301,8 +299,6 @@ int h2o_create_ex(int B, int Hq, int Hkv, int d, int C, int dtype, int max_T, h2
         return bail(cuda_fail(c, e, "cudaMalloc(scores)"));
     if ((e = cudaMalloc(&c->pos, sizeof(int32_t) * groups * C)) != cudaSuccess)
         return bail(cuda_fail(c, e, "cudaMalloc(positions)"));
-    if ((e = cudaMalloc(&c->free_list, sizeof(int32_t) * groups * C)) != cudaSuccess)
-        return bail(cuda_fail(c, e, "cudaMalloc(free_list)"));
     int rc = alloc_workspace(c, max_T);
     if (rc != H2O_OK) return bail(rc);
     if ((e = cudaHostAlloc((void**)&c->err_host, sizeof(int), cudaHostAllocMapped)) != cudaSuccess)
@@ -333,7 +329,6 @@ int h2o_destroy(h2o_ctx* c) {
     cudaFree(c->Vc);
     cudaFree(c->scores);
     cudaFree(c->pos);
-    cudaFree(c->free_list);
     cudaFree(c->stage);
     if (c->err_host) cudaFreeHost(c->err_host);
     delete c;

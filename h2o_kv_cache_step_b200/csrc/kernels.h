@@ -45,7 +45,6 @@ struct StepArgs {
     int32_t* cand_pos;   // [B,Hkv,C+tmax]
     uint8_t* cand_kept;  // [B,Hkv,C+tmax]
     int32_t* token_slot; // [B,Hkv,tmax]
-    int32_t* free_list;  // [B,Hkv,C]
     float* partials;     // weight-sum partials [nparts][B*Hkv][C+tmax] (tensor-core path)
     size_t partial_elems;
     int nparts;          // > 0: the selection kernel first sums the partials

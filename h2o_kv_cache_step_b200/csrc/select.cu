@@ -90,7 +90,7 @@ template <bool SMEM_KEYS>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
               uint8_t* __restrict__ cand_kept, int32_t* __restrict__ token_slot,
-              int32_t* __restrict__ free_list, float* __restrict__ scores, int32_t* __restrict__ pos,
+              float* __restrict__ scores, int32_t* __restrict__ pos,
               const float* __restrict__ partials, int nparts, int C, int T, int n, int tmax, long long P,
               int policy) {
     __shared__ unsigned int hist[256];
@@ -405,11 +405,11 @@ cudaError_t launch_select(const StepArgs& a) {
     cudaError_t e;
     if (with_keys <= (size_t)kSelectSmemLimit) {
         e = launch_ex(kEarlyLaunch, select_kernel<true>, dim3(a.B * a.Hkv), dim3(kSelThreads), with_keys, a.stream, a.cand_score,
-                       a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
+                       a.cand_pos, a.cand_kept, a.token_slot, a.scores, a.pos, (const float*)a.partials,
                        a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P, a.policy);
     } else if (tail <= (size_t)kSelectSmemLimit) {
         e = launch_ex(kEarlyLaunch, select_kernel<false>, dim3(a.B * a.Hkv), dim3(kSelThreads), tail, a.stream, a.cand_score,
-                       a.cand_pos, a.cand_kept, a.token_slot, a.free_list, a.scores, a.pos, (const float*)a.partials,
+                       a.cand_pos, a.cand_kept, a.token_slot, a.scores, a.pos, (const float*)a.partials,
                        a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P, a.policy);
     } else {
         return cudaErrorInvalidConfiguration;

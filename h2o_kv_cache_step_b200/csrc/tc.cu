@@ -44,7 +44,6 @@ using tc::ex2;
 using tc::fence_after_sync;
 using tc::fence_before_sync;
 
-constexpr int kThreads = 192;
 // P may exceed 1 by up to 2^16 before the running maximum is moved: P is
 // bf16 (same exponent range as fp32) and O and the row sum accumulate in fp32,
 // so only overflow matters, and this keeps far from it.
