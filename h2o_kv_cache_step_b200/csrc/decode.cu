@@ -206,13 +206,9 @@ cudaError_t launch_decode_typed(const StepArgs& a) {
     const int nsplit = (a.n + kDecodeSplit - 1) / kDecodeSplit + 1;
     const int lstride = a.C + kDecodeMaxT;
     const size_t smem = DecSmem<D>::bytes(R);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)DecSmem<D>::bytes(kDecodeMaxRows));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    if (cudaError_t e = ensure_smem_limit(decode_split_kernel<E, D>, (int)DecSmem<D>::bytes(kDecodeMaxRows));
+        e != cudaSuccess)
+        return e;
     const float scale_log2 = kLog2e / sqrtf((float)D);
     cudaError_t e = launch_ex(true, decode_split_kernel<E, D>, dim3(nsplit, groups), dim3(kDecThreads), smem,
                               a.stream, (const E*)a.q, (const E*)a.k, (const E*)a.v, (const E*)a.Kc,

@@ -4,6 +4,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "common.cuh"
 
 namespace h2o {
@@ -89,6 +93,23 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     const bool pdl = false;  // measured: no gain for the tensor-core kernels
 #endif
     return launch_ex(pdl, kernel, grid, block, smem, stream, args...);
+}
+
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device); safe to call from several threads.
+template <typename... KArgs>
+cudaError_t ensure_smem_limit(void (*kernel)(KArgs...), int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::set<std::pair<const void*, int>> done;
+    const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count(key)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert(key);
+    return e;
 }
 
 // SIMT kernels (fp32 path; any supported d).

@@ -393,15 +393,8 @@ cudaError_t launch_select(const StepArgs& a) {
     const int m = a.n + a.T;
     const size_t tail = (((size_t)m + 15) & ~(size_t)15) + (size_t)a.C * 4;  // kept flags + free list
     const size_t with_keys = (size_t)m * 8 + tail;
-    static int configured = 0;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSelectSmemLimit);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmemLimit);
-        if (e != cudaSuccess) return e;
-        configured = 1;
-    }
+    if (cudaError_t e = ensure_smem_limit(select_kernel<true>, kSelectSmemLimit); e != cudaSuccess) return e;
+    if (cudaError_t e = ensure_smem_limit(select_kernel<false>, kSelectSmemLimit); e != cudaSuccess) return e;
     cudaError_t e;
     if (with_keys <= (size_t)kSelectSmemLimit) {
         e = launch_ex(kEarlyLaunch, select_kernel<true>, dim3(a.B * a.Hkv), dim3(kSelThreads), with_keys, a.stream, a.cand_score,

@@ -191,7 +191,7 @@ cudaError_t wsum_simt_typed(const StepArgs& a) {
     dim3 grid((n_cand + kKeysPerBlock - 1) / kKeysPerBlock, a.Hkv, a.B);
     const size_t smem = sizeof(float) * (kKeysPerBlock * (D + 1) + kRowTile * D + kRowTile);
     auto kern = wsum_simt_kernel<E, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_limit(kern, (int)smem);
     if (e != cudaSuccess) return e;
     const float scale_log2 = kLog2e / sqrtf((float)D);
     kern<<<grid, kKeysPerBlock, smem, a.stream>>>(

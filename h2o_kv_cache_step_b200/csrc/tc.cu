@@ -850,12 +850,7 @@ int nparts_for(int G, int T) { return (G * T + kRowsPerUnit - 1) / kRowsPerUnit;
 template <int D>
 cudaError_t sdpa_launch(const StepArgs& a) {
     using Cfg = SdpaCfg<D>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(sdpa_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    if (cudaError_t e = ensure_smem_limit(sdpa_tc_kernel<D>, Cfg::SMEM); e != cudaSuccess) return e;
     CUtensorMap mq, mkc, mvc, mk, mv;
     if (!make_map(&mq, a.q, (uint64_t)a.B * a.Hq * a.T, D) || !make_map(&mkc, a.Kc, (uint64_t)a.B * a.Hkv * a.C, D) ||
         !make_map(&mvc, a.Vc, (uint64_t)a.B * a.Hkv * a.C, D) || !make_map(&mk, a.k, (uint64_t)a.B * a.Hkv * a.T, D) ||
@@ -889,12 +884,7 @@ cudaError_t sdpa_launch(const StepArgs& a) {
 template <int D>
 cudaError_t wsum_launch(const StepArgs& a) {
     using Cfg = WsumCfg<D>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(wsum_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    if (cudaError_t e = ensure_smem_limit(wsum_tc_kernel<D>, Cfg::SMEM); e != cudaSuccess) return e;
     const int G = a.Hq / a.Hkv;
     const int groups = a.B * a.Hkv;
     const int n_ru = (G * a.T + kRowsPerUnit - 1) / kRowsPerUnit;
