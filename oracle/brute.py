@@ -24,12 +24,16 @@ class BruteH2O:
     cache[b][g] maps position -> [key (d,), value (d,), score].
     """
 
-    def __init__(self, B: int, Hq: int, Hkv: int, d: int, C: int, normalized: bool = False):
+    def __init__(self, B: int, Hq: int, Hkv: int, d: int, C: int, normalized: bool = False,
+                 insert_always: bool = False):
         """normalized: rank eviction candidates by score / age (age = token
         count after the step minus the position, the same section's improved
         score) instead of by the score."""
         self.B, self.Hq, self.Hkv, self.d, self.C = B, Hq, Hkv, d, C
         self.normalized = normalized
+        # insert_always: evict the lowest-scoring entries before the chunk
+        # attends (by the scores so far), so every chunk token enters
+        self.insert_always = insert_always
         self.G = Hq // Hkv
         self.P = 0
         self.cache = [[dict() for _ in range(Hkv)] for _ in range(B)]
@@ -50,6 +54,11 @@ class BruteH2O:
             kept_sets.append([])
             for g in range(self.Hkv):
                 old = self.cache[b][g]
+                if self.insert_always:
+                    extra = len(old) + T - self.C
+                    if extra > 0:
+                        lowest = sorted(old, key=lambda p: (old[p][2], p))[:extra]
+                        old = {p: e for p, e in old.items() if p not in lowest}
                 cand = {p: [e[0], e[1], e[2]] for p, e in old.items()}
                 for t in range(T):
                     cand[self.P + t] = [k[b, g, t], v[b, g, t], 0.0]
@@ -74,7 +83,7 @@ class BruteH2O:
                 t_now = self.P + T
                 rank = (lambda p: cand[p][2] / (t_now - p)) if self.normalized else (lambda p: cand[p][2])
                 order = sorted(positions, key=lambda p: (rank(p), p), reverse=True)
-                keep = set(order[: self.C])
+                keep = set(order[: self.C]) if not self.insert_always else set(positions)
                 kept_sets[b].append(keep)
                 self.cache[b][g] = {p: cand[p] for p in keep}
         self.P += T

@@ -33,6 +33,9 @@
  *     age is at least 1 (the page's superscript is garbled; this is the
  *     plainest reading).
  *
+ * h2o_oracle_step_insert is the insert-always variant of the same section
+ * (evict before the chunk attends, every chunk token enters; see there).
+ *
  * Everything is fp64, plain loops, exp()/log() from libm. OpenMP only splits
  * independent (batch, KV head) groups or independent query rows; no result
  * depends on the thread count.
@@ -299,6 +302,116 @@ int h2o_oracle_step(int B, int Hq, int Hkv, int d, int C, int T, int64_t P,
     return h2o_oracle_step_policy(B, Hq, Hkv, d, C, T, P, 0, Kc, Vc, phi, pos, q, k, v, out, lse,
                                   cand_score, cand_pos, cand_slot, cand_kept, n_cand, token_slot,
                                   nthreads);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Insert-always variant ("Learning how to Forget", paper page, section
+ * "Improvements to Heavy-Hitter Oracle (H2O)": new content overwrites the
+ * slots with the smallest scores; section "Kernel Support Needs": attention
+ * under the position mask). Reading taken: before the chunk attends, if the
+ * cache cannot hold the n valid entries plus the T chunk tokens, the
+ * n + T - C valid slots with the lowest pre-step scores are evicted (lowest
+ * score first, the older position first among equal scores); the chunk
+ * tokens, in position order, fill the empty and evicted slots in ascending
+ * slot order with score 0; then every row attends to the C-slot buffer,
+ * slot j visible to row i iff pos(j) <= P + i, and every valid slot's score
+ * grows by the weights it receives. No chunk token is dropped, so T <= C. */
+static int group_step_insert(int G, int d, int C, int T, int64_t P,
+                             double *Kc, double *Vc, double *phi, int64_t *pos,
+                             const double *q, const double *k, const double *v,
+                             double *out, double *lse, int32_t *token_slot)
+{
+    if (T > C) return ORACLE_ERR_ARG;
+    const double scale = 1.0 / sqrt((double)d);
+    int n = 0;
+    for (int j = 0; j < C; ++j) n += pos[j] >= 0;
+    const int need = n + T - C;  /* valid slots to evict, if positive */
+    uint8_t *evict = (uint8_t *)calloc((size_t)C, 1);
+    double *w = (double *)malloc(sizeof(double) * (size_t)C);
+    double *delta = (double *)calloc((size_t)C, sizeof(double));
+    if (!evict || !w || !delta) { free(evict); free(w); free(delta); return ORACLE_ERR_OOM; }
+    /* a valid slot goes iff fewer than `need` valid slots rank below it */
+    for (int a = 0; need > 0 && a < C; ++a) {
+        if (pos[a] < 0) continue;
+        int below = 0;
+        for (int b = 0; b < C; ++b)
+            if (b != a && pos[b] >= 0 && ranks_above(phi[a], pos[a], phi[b], pos[b])) ++below;
+        evict[a] = (uint8_t)(below < need);
+    }
+    /* free slots (empty or evicted) in ascending order take the chunk tokens */
+    int t = 0;
+    for (int j = 0; j < C && t < T; ++j) {
+        if (pos[j] >= 0 && !evict[j]) continue;
+        memcpy(Kc + (size_t)j * d, k + (size_t)t * d, sizeof(double) * (size_t)d);
+        memcpy(Vc + (size_t)j * d, v + (size_t)t * d, sizeof(double) * (size_t)d);
+        phi[j] = 0.0;
+        pos[j] = P + t;
+        token_slot[t] = j;
+        ++t;
+    }
+    for (int j = 0; j < C; ++j)  /* evicted slots no chunk token took */
+        if (evict[j] && pos[j] < P) { pos[j] = -1; phi[j] = 0.0; }
+    /* attention over the buffer under the position mask */
+    for (int h = 0; h < G; ++h) {
+        for (int i = 0; i < T; ++i) {
+            const double *qrow = q + ((size_t)h * T + i) * d;
+            double m = -INFINITY;
+            for (int j = 0; j < C; ++j) {
+                if (pos[j] < 0 || pos[j] > P + i) continue;
+                w[j] = logit(qrow, Kc + (size_t)j * d, d, scale);
+                if (w[j] > m) m = w[j];
+            }
+            double Z = 0.0;
+            for (int j = 0; j < C; ++j)
+                if (pos[j] >= 0 && pos[j] <= P + i) Z += exp(w[j] - m);
+            double *orow = out + ((size_t)h * T + i) * d;
+            for (int x = 0; x < d; ++x) orow[x] = 0.0;
+            for (int j = 0; j < C; ++j) {
+                if (pos[j] < 0 || pos[j] > P + i) continue;
+                const double wj = exp(w[j] - m) / Z;
+                for (int x = 0; x < d; ++x) orow[x] += wj * Vc[(size_t)j * d + x];
+                delta[j] += wj;
+            }
+            lse[(size_t)h * T + i] = m + log(Z);
+        }
+    }
+    for (int j = 0; j < C; ++j)
+        if (pos[j] >= 0) phi[j] += delta[j];
+    free(evict); free(w); free(delta);
+    return ORACLE_OK;
+}
+
+/* The insert-always step for the whole batch (layouts as h2o_oracle_step;
+ * token_slot [B,Hkv,T] receives each chunk token's slot). */
+int h2o_oracle_step_insert(int B, int Hq, int Hkv, int d, int C, int T, int64_t P,
+                           double *Kc, double *Vc, double *phi, int64_t *pos,
+                           const double *q, const double *k, const double *v,
+                           double *out, double *lse, int32_t *token_slot, int nthreads)
+{
+    if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0 || d <= 0 || C <= 0 || T <= 0 || T > C || P < 0)
+        return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    const int groups = B * Hkv;
+    int rc_all = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int bg = 0; bg < groups; ++bg) {
+        const int b = bg / Hkv, g = bg % Hkv;
+        const size_t cs = (size_t)bg * C;
+        const size_t qo = ((size_t)b * Hq + (size_t)g * G) * T;
+        int rc = group_step_insert(G, d, C, T, P, Kc + cs * d, Vc + cs * d, phi + cs, pos + cs,
+                                   q + qo * d, k + (size_t)bg * T * d, v + (size_t)bg * T * d,
+                                   out + qo * d, lse + qo, token_slot + (size_t)bg * T);
+        if (rc != ORACLE_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            rc_all = rc;
+        }
+    }
+    return rc_all;
 }
 
 /*

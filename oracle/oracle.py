@@ -47,6 +47,8 @@ def lib():
         L.h2o_oracle_step.restype = I
         L.h2o_oracle_step_policy.argtypes = [I, I, I, I, I, I, ctypes.c_int64, I] + [P] * 15 + [I]
         L.h2o_oracle_step_policy.restype = I
+        L.h2o_oracle_step_insert.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 10 + [I]
+        L.h2o_oracle_step_insert.restype = I
         L.h2o_oracle_select_group.argtypes = [I, I, I, P, P, P, P, P]
         L.h2o_oracle_select_group.restype = I
         L.h2o_oracle_rows.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 6 + [I, P, P, P, I]
@@ -130,6 +132,30 @@ def step(state: State, q: np.ndarray, k: np.ndarray, v: np.ndarray, nthreads: in
         raise RuntimeError(f"h2o_oracle_step failed: {rc}")
     state.P += T
     return StepResult(out, lse, cs, cp, cslot, ck, nc, ts)
+
+
+def step_insert_always(state: State, q: np.ndarray, k: np.ndarray, v: np.ndarray, nthreads: int = 0):
+    """The insert-always variant of the step (T <= C): evict the lowest-scoring
+    valid slots first if the chunk does not fit, write the chunk into the
+    free slots, then attend over the buffer under the position mask and add
+    the weights to the scores. Mutates ``state``; returns (out, lse,
+    token_slot)."""
+    q = np.ascontiguousarray(q, np.float64)
+    k = np.ascontiguousarray(k, np.float64)
+    v = np.ascontiguousarray(v, np.float64)
+    B, Hq, T, d = q.shape
+    _, Hkv, C, _ = state.K.shape
+    assert k.shape == (B, Hkv, T, d) and v.shape == (B, Hkv, T, d)
+    out = np.zeros((B, Hq, T, d))
+    lse = np.zeros((B, Hq, T))
+    ts = np.full((B, Hkv, T), -1, np.int32)
+    rc = lib().h2o_oracle_step_insert(B, Hq, Hkv, d, C, T, int(state.P),
+                                      _p(state.K), _p(state.V), _p(state.phi), _p(state.pos),
+                                      _p(q), _p(k), _p(v), _p(out), _p(lse), _p(ts), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"h2o_oracle_step_insert failed: {rc}")
+    state.P += T
+    return out, lse, ts
 
 
 def select_group(C: int, T: int, cand_score, cand_pos, cand_slot):

@@ -271,3 +271,86 @@ def test_select_against_sort_with_planted_ties(oracle_lib, seed):
     placed = [int(ts[t]) for t in range(T) if kept[n_valid + t]]
     assert placed == free[: len(placed)]
     assert all(ts[t] == -1 for t in range(T) if not kept[n_valid + t])
+
+
+# ------------------------------------------------------- insert-always ---
+def test_insert_always_hand_worked_example(oracle_lib):
+    g = json.load(open(os.path.join(GOLDEN, "worked_example_c3_t2_insert_always.json")))
+    s = g["shape"]
+    st = oracle.State.empty(s["B"], s["Hkv"], s["C"], s["d"])
+    T = s["T"]
+    for ch in g["chunks"]:
+        q = np.array([_val(x) for x in ch["q"]]).reshape(1, 1, T, 1)
+        k = np.array([_val(x) for x in ch["k"]]).reshape(1, 1, T, 1)
+        v = np.array([_val(x) for x in ch["v"]]).reshape(1, 1, T, 1)
+        out, lse, ts = oracle.step_insert_always(st, q, k, v)
+        np.testing.assert_allclose(out.ravel(), [_val(x) for x in ch["out"]], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse.ravel(), [_val(x) for x in ch["lse"]], rtol=0, atol=1e-13)
+        assert ts[0, 0].tolist() == ch["token_slot"]
+        assert st.pos[0, 0].tolist() == ch["slot_pos"]
+        np.testing.assert_allclose(st.phi[0, 0], [_val(x) for x in ch["slot_score"]], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,C,T,n_chunks,kscale", [
+    (2, 4, 2, 8, 6, 3, 5, 1.0),     # GQA groups of 2
+    (1, 2, 1, 5, 4, 1, 9, 2.0),     # T = 1
+    (1, 3, 3, 4, 5, 5, 3, 1.5),     # T = C: the whole cache turns over every step
+    (1, 4, 1, 6, 7, 4, 4, 0.5),     # G = 4
+])
+def test_insert_always_matches_brute_force(oracle_lib, B, Hq, Hkv, d, C, T, n_chunks, kscale):
+    gen = iid_gen(B, Hq, Hkv, d, T, seed=C * 7 + T, kscale=kscale)
+    st = oracle.State.empty(B, Hkv, C, d)
+    br = brute.BruteH2O(B, Hq, Hkv, d, C, insert_always=True)
+    for c in range(n_chunks):
+        q, k, v = gen(c)
+        out, lse, ts = oracle.step_insert_always(st, q, k, v)
+        bo, bl, bs, bk = br.step(q, k, v)
+        np.testing.assert_allclose(out, bo, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, bl, rtol=0, atol=1e-12)
+        for b in range(B):
+            for g in range(Hkv):
+                valid = st.pos[b, g] >= 0
+                assert set(st.pos[b, g][valid].tolist()) == bk[b][g]
+                for slot in np.nonzero(valid)[0]:
+                    assert abs(st.phi[b, g, slot] - bs[b][g][int(st.pos[b, g, slot])]) <= 1e-12
+                # every chunk token entered, at the slot it reports
+                P0 = st.P - T
+                assert np.array_equal(st.pos[b, g, ts[b, g]], P0 + np.arange(T))
+
+
+def test_insert_always_equals_the_step_while_nothing_is_evicted(oracle_lib):
+    """With room for every chunk (n + T <= C) both orders give the same
+    outputs, scores and slots: nothing is evicted before or after."""
+    B, Hq, Hkv, d, C, T = 1, 4, 2, 8, 40, 6
+    gen = iid_gen(B, Hq, Hkv, d, T, seed=77)
+    a, b = oracle.State.empty(B, Hkv, C, d), oracle.State.empty(B, Hkv, C, d)
+    for c in range(C // T):
+        q, k, v = gen(c)
+        out, lse, ts = oracle.step_insert_always(a, q, k, v)
+        r = oracle.step(b, q, k, v)
+        np.testing.assert_allclose(out, r.out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, r.lse, rtol=0, atol=1e-12)
+        assert np.array_equal(ts, r.token_slot)
+        assert np.array_equal(a.pos, b.pos)
+        np.testing.assert_allclose(a.phi, b.phi, rtol=0, atol=1e-12)
+
+
+def test_insert_always_score_mass_and_rejects_long_chunks(oracle_lib):
+    """Each row's weights sum to one, so a step adds G*T of score per group
+    (over the slots that survive it); a chunk longer than the cache is an
+    argument error for this variant."""
+    B, Hq, Hkv, d, C, T = 1, 6, 2, 4, 5, 3
+    gen = iid_gen(B, Hq, Hkv, d, T, seed=5)
+    st = oracle.State.empty(B, Hkv, C, d)
+    for c in range(4):
+        q, k, v = gen(c)
+        before = st.phi.copy()
+        pos_before = st.pos.copy()
+        oracle.step_insert_always(st, q, k, v)
+        for g in range(Hkv):
+            kept_old = [j for j in range(C) if pos_before[0, g, j] >= 0 and st.pos[0, g, j] == pos_before[0, g, j]]
+            mass = st.phi[0, g].sum() - before[0, g, kept_old].sum()
+            assert abs(mass - (Hq // Hkv) * T) < 1e-12
+    q, k, v = iid_gen(B, Hq, Hkv, d, C + 1, seed=6)(0)
+    with pytest.raises(RuntimeError):
+        oracle.step_insert_always(oracle.State.empty(B, Hkv, C, d), q, k, v)
