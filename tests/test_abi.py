@@ -72,3 +72,17 @@ def test_create_without_gpu_fails_cleanly(L):
     assert rc in (_lib.H2O_ERR_CUDA, _lib.H2O_ERR_OOM)
     assert not h.value
     assert b"cuda" in L.h2o_last_error(None).lower()
+
+
+def test_new_entry_points_reject_a_null_context(L):
+    assert L.h2o_set_policy(None, _lib.H2O_POLICY_SUM) == _lib.H2O_ERR_ARG
+    assert L.h2o_host_sync(None) == _lib.H2O_ERR_ARG
+    assert L.h2o_step_host_async(None, None, None, None, None, 4, None) == _lib.H2O_ERR_ARG
+    assert L.h2o_last_error(None)
+
+
+def test_policy_constants_match_the_header():
+    src = open(os.path.join(ROOT, "include", "h2o.h")).read()
+    m = re.search(r"enum h2o_policy \{\s*H2O_POLICY_SUM = (\d+),\s*H2O_POLICY_NORMALIZED = (\d+)\s*\}", src)
+    assert m, "enum h2o_policy not found in h2o.h"
+    assert (int(m.group(1)), int(m.group(2))) == (_lib.H2O_POLICY_SUM, _lib.H2O_POLICY_NORMALIZED)
