@@ -35,6 +35,9 @@
  *
  * h2o_oracle_step_insert is the insert-always variant of the same section
  * (evict before the chunk attends, every chunk token enters; see there).
+ * h2o_oracle_backward is the gradient of the chunk SDPA with the kept set
+ * fixed (the paper's fine-tuning trains through the sparse cache; the
+ * eviction itself is replayed, not differentiated).
  *
  * Everything is fp64, plain loops, exp()/log() from libm. OpenMP only splits
  * independent (batch, KV head) groups or independent query rows; no result
@@ -404,6 +407,111 @@ int h2o_oracle_step_insert(int B, int Hq, int Hkv, int d, int C, int T, int64_t 
         int rc = group_step_insert(G, d, C, T, P, Kc + cs * d, Vc + cs * d, phi + cs, pos + cs,
                                    q + qo * d, k + (size_t)bg * T * d, v + (size_t)bg * T * d,
                                    out + qo * d, lse + qo, token_slot + (size_t)bg * T);
+        if (rc != ORACLE_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            rc_all = rc;
+        }
+    }
+    return rc_all;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the chunk SDPA with the kept set fixed (the eviction is a
+ * discrete choice, replayed, not differentiated): given dL/dO, the gradients
+ * of L with respect to q, the chunk's k and v, and the cache's K and V, for
+ * the same key set and mask as the forward (valid cache slots all visible,
+ * chunk token t visible to row i iff t <= i), scale 1/sqrt(d). Per row:
+ *   p = softmax(s), s_j = scale q.k_j;  dv_j += p_j dO;  dp_j = dO.v_j;
+ *   ds_j = p_j (dp_j - sum_l p_l dp_l);  dq = scale sum_j ds_j k_j;
+ *   dk_j += scale ds_j q.
+ * Gradients of one KV head sum over the query heads of its group. Empty
+ * cache slots get zero gradients. */
+static int group_backward(int G, int d, int C, int T, int64_t P,
+                          const double *Kc, const double *Vc, const int64_t *pos,
+                          const double *q, const double *k, const double *v, const double *dout,
+                          double *dq, double *dKc, double *dVc, double *dk, double *dv)
+{
+    const double scale = 1.0 / sqrt((double)d);
+    const int nk = C + T;  /* key index j: cache slot j < C, chunk token j - C */
+    double *p = (double *)malloc(sizeof(double) * (size_t)nk);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)nk);
+    if (!p || !dp) { free(p); free(dp); return ORACLE_ERR_OOM; }
+    memset(dKc, 0, sizeof(double) * (size_t)C * d);
+    memset(dVc, 0, sizeof(double) * (size_t)C * d);
+    memset(dk, 0, sizeof(double) * (size_t)T * d);
+    memset(dv, 0, sizeof(double) * (size_t)T * d);
+    for (int h = 0; h < G; ++h) {
+        for (int i = 0; i < T; ++i) {
+            const double *qrow = q + ((size_t)h * T + i) * d;
+            const double *go = dout + ((size_t)h * T + i) * d;
+            double *gq = dq + ((size_t)h * T + i) * d;
+            double m = -INFINITY;
+            for (int j = 0; j < nk; ++j) {
+                const int vis = j < C ? pos[j] >= 0 : (j - C) <= i;
+                if (!vis) { p[j] = -INFINITY; continue; }
+                const double *kr = j < C ? Kc + (size_t)j * d : k + (size_t)(j - C) * d;
+                p[j] = logit(qrow, kr, d, scale);
+                if (p[j] > m) m = p[j];
+            }
+            double Z = 0.0;
+            for (int j = 0; j < nk; ++j)
+                if (p[j] != -INFINITY) Z += exp(p[j] - m);
+            double pdp = 0.0;
+            for (int j = 0; j < nk; ++j) {
+                if (p[j] == -INFINITY) { p[j] = 0.0; dp[j] = 0.0; continue; }
+                p[j] = exp(p[j] - m) / Z;
+                const double *vr = j < C ? Vc + (size_t)j * d : v + (size_t)(j - C) * d;
+                double acc = 0.0;
+                for (int x = 0; x < d; ++x) acc += go[x] * vr[x];
+                dp[j] = acc;
+                pdp += p[j] * acc;
+            }
+            for (int x = 0; x < d; ++x) gq[x] = 0.0;
+            for (int j = 0; j < nk; ++j) {
+                if (p[j] == 0.0 && dp[j] == 0.0) continue;
+                const double ds = p[j] * (dp[j] - pdp);
+                const double *kr = j < C ? Kc + (size_t)j * d : k + (size_t)(j - C) * d;
+                double *gk = j < C ? dKc + (size_t)j * d : dk + (size_t)(j - C) * d;
+                double *gv = j < C ? dVc + (size_t)j * d : dv + (size_t)(j - C) * d;
+                for (int x = 0; x < d; ++x) {
+                    gq[x] += scale * ds * kr[x];
+                    gk[x] += scale * ds * qrow[x];
+                    gv[x] += p[j] * go[x];
+                }
+            }
+        }
+    }
+    (void)P;
+    free(p); free(dp);
+    return ORACLE_OK;
+}
+
+/* Backward for the whole batch. Layouts: as h2o_oracle_step for Kc, Vc, pos,
+ * q, k, v; dout and dq [B,Hq,T,d]; dKc, dVc [B,Hkv,C,d]; dk, dv [B,Hkv,T,d]. */
+int h2o_oracle_backward(int B, int Hq, int Hkv, int d, int C, int T, int64_t P,
+                        const double *Kc, const double *Vc, const int64_t *pos,
+                        const double *q, const double *k, const double *v, const double *dout,
+                        double *dq, double *dKc, double *dVc, double *dk, double *dv, int nthreads)
+{
+    if (B <= 0 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0 || d <= 0 || C <= 0 || T <= 0 || P < 0)
+        return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    const int groups = B * Hkv;
+    int rc_all = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int bg = 0; bg < groups; ++bg) {
+        const int b = bg / Hkv, g = bg % Hkv;
+        const size_t cs = (size_t)bg * C;
+        const size_t qo = ((size_t)b * Hq + (size_t)g * G) * T;
+        int rc = group_backward(G, d, C, T, P, Kc + cs * d, Vc + cs * d, pos + cs,
+                                q + qo * d, k + (size_t)bg * T * d, v + (size_t)bg * T * d, dout + qo * d,
+                                dq + qo * d, dKc + cs * d, dVc + cs * d, dk + (size_t)bg * T * d,
+                                dv + (size_t)bg * T * d);
         if (rc != ORACLE_OK) {
 #ifdef _OPENMP
 #pragma omp critical

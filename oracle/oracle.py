@@ -49,6 +49,8 @@ def lib():
         L.h2o_oracle_step_policy.restype = I
         L.h2o_oracle_step_insert.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 10 + [I]
         L.h2o_oracle_step_insert.restype = I
+        L.h2o_oracle_backward.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 12 + [I]
+        L.h2o_oracle_backward.restype = I
         L.h2o_oracle_select_group.argtypes = [I, I, I, P, P, P, P, P]
         L.h2o_oracle_select_group.restype = I
         L.h2o_oracle_rows.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 6 + [I, P, P, P, I]
@@ -156,6 +158,26 @@ def step_insert_always(state: State, q: np.ndarray, k: np.ndarray, v: np.ndarray
         raise RuntimeError(f"h2o_oracle_step_insert failed: {rc}")
     state.P += T
     return out, lse, ts
+
+
+def backward(state: State, q, k, v, dout, nthreads: int = 0):
+    """Gradients of sum(dout * O) for one step's SDPA with the kept set fixed:
+    returns dq [B,Hq,T,d], dKc, dVc [B,Hkv,C,d] (zero for empty slots) and
+    dk, dv [B,Hkv,T,d]. ``state`` is the cache before the step (unchanged)."""
+    q, k, v, dout = (np.ascontiguousarray(x, np.float64) for x in (q, k, v, dout))
+    B, Hq, T, d = q.shape
+    _, Hkv, C, _ = state.K.shape
+    dq = np.zeros_like(q)
+    dKc = np.zeros_like(state.K)
+    dVc = np.zeros_like(state.V)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    rc = lib().h2o_oracle_backward(B, Hq, Hkv, d, C, T, int(state.P), _p(state.K), _p(state.V), _p(state.pos),
+                                   _p(q), _p(k), _p(v), _p(dout), _p(dq), _p(dKc), _p(dVc), _p(dk), _p(dv),
+                                   int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"h2o_oracle_backward failed: {rc}")
+    return dq, dKc, dVc, dk, dv
 
 
 def select_group(C: int, T: int, cand_score, cand_pos, cand_slot):

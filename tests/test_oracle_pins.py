@@ -354,3 +354,90 @@ def test_insert_always_score_mass_and_rejects_long_chunks(oracle_lib):
     q, k, v = iid_gen(B, Hq, Hkv, d, C + 1, seed=6)(0)
     with pytest.raises(RuntimeError):
         oracle.step_insert_always(oracle.State.empty(B, Hkv, C, d), q, k, v)
+
+
+# ------------------------------------------------------------- backward ---
+def _backward_case(seed, B=1, Hq=4, Hkv=2, d=3, C=5, n=3, T=3, vconst=False):
+    r = np.random.default_rng(seed)
+    st = oracle.State.empty(B, Hkv, C, d)
+    st.K[:, :, :n] = r.standard_normal((B, Hkv, n, d))
+    st.V[:, :, :n] = r.standard_normal((B, Hkv, n, d))
+    st.pos[:, :, :n] = np.arange(n)
+    st.P = n + 2
+    q = r.standard_normal((B, Hq, T, d))
+    k = r.standard_normal((B, Hkv, T, d))
+    v = r.standard_normal((B, Hkv, T, d))
+    if vconst:
+        st.V[:, :, :n] = 0.7
+        v[:] = 0.7
+    dout = r.standard_normal((B, Hq, T, d))
+    return st, q, k, v, dout
+
+
+def _loss(st, q, k, v, dout):
+    return float((oracle.step(st.copy(), q, k, v).out * dout).sum())
+
+
+def test_backward_matches_finite_differences(oracle_lib):
+    st, q, k, v, dout = _backward_case(1)
+    dq, dKc, dVc, dk, dv = oracle.backward(st, q, k, v, dout)
+    eps = 1e-6
+    n = int(st.n_valid[0, 0])
+    checks = [("q", q, dq), ("k", k, dk), ("v", v, dv)]
+    for name, arr, grad in checks:
+        for idx in np.ndindex(arr.shape):
+            a = arr.copy(); a[idx] += eps
+            b = arr.copy(); b[idx] -= eps
+            args = {"q": q, "k": k, "v": v}
+            lp = _loss(st, **{**args, name: a}, dout=dout)
+            lm = _loss(st, **{**args, name: b}, dout=dout)
+            assert abs((lp - lm) / (2 * eps) - grad[idx]) < 1e-7, (name, idx)
+    for name, grad in (("K", dKc), ("V", dVc)):
+        for idx in np.ndindex(getattr(st, name).shape):
+            if idx[2] >= n:
+                assert grad[idx] == 0.0  # empty slot
+                continue
+            sp, sm = st.copy(), st.copy()
+            getattr(sp, name)[idx] += eps
+            getattr(sm, name)[idx] -= eps
+            fd = (_loss(sp, q, k, v, dout) - _loss(sm, q, k, v, dout)) / (2 * eps)
+            assert abs(fd - grad[idx]) < 1e-7, (name, idx)
+
+
+def test_backward_matches_torch_autograd(oracle_lib):
+    import torch
+    st, q, k, v, dout = _backward_case(2, B=2, Hq=6, Hkv=3, d=5, C=7, n=6, T=4)
+    dq, dKc, dVc, dk, dv = oracle.backward(st, q, k, v, dout)
+    B, Hq, T, d = q.shape
+    Hkv, C, G = k.shape[1], st.K.shape[2], q.shape[1] // k.shape[1]
+    tq = torch.tensor(q, requires_grad=True)
+    tk = torch.tensor(k, requires_grad=True)
+    tv = torch.tensor(v, requires_grad=True)
+    tK = torch.tensor(st.K, requires_grad=True)
+    tV = torch.tensor(st.V, requires_grad=True)
+    loss = torch.zeros((), dtype=torch.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            valid = [j for j in range(C) if st.pos[b, g, j] >= 0]
+            for i in range(T):
+                keys = torch.cat([tK[b, g, valid], tk[b, g, : i + 1]])
+                vals = torch.cat([tV[b, g, valid], tv[b, g, : i + 1]])
+                w = torch.softmax(keys @ tq[b, h, i] / np.sqrt(d), dim=0)
+                loss = loss + (w @ vals * torch.tensor(dout[b, h, i])).sum()
+    loss.backward()
+    for ours, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad), (dKc, tK.grad), (dVc, tV.grad)):
+        np.testing.assert_allclose(ours, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_equal_values_give_no_query_or_key_gradient(oracle_lib):
+    """With every visible value row equal, O does not depend on the weights:
+    dq, dk and the cache's dK vanish; dV still receives the weights times dO."""
+    st, q, k, v, dout = _backward_case(3, vconst=True)
+    dq, dKc, dVc, dk, dv = oracle.backward(st, q, k, v, dout)
+    assert np.abs(dq).max() < 1e-14 and np.abs(dk).max() < 1e-14 and np.abs(dKc).max() < 1e-14
+    # every row's weights sum to one, so the value gradients add up to sum of dO per KV head
+    G = q.shape[1] // k.shape[1]
+    for g in range(k.shape[1]):
+        total = dVc[0, g].sum(axis=0) + dv[0, g].sum(axis=0)
+        np.testing.assert_allclose(total, dout[0, g * G:(g + 1) * G].sum(axis=(0, 1)), rtol=0, atol=1e-12)
