@@ -1,0 +1,51 @@
+"""Host-side logic of bench.py that the GPU runs rely on (no GPU needed)."""
+import os
+import shutil
+
+import pytest
+
+import bench
+from h2o_kv_cache_step_b200 import synth
+
+WL = synth.WORKLOADS["qwen3-4b-c2048-t1024-n64k"]
+
+
+def test_schedule_fills_then_stays_full():
+    sched = bench.sequence_schedule(WL)
+    assert len(sched) == WL.n_chunks
+    assert sched[:3] == [(0, WL.T), (WL.T, WL.T), (2 * WL.T, WL.T)]
+    assert all(n == WL.C for n, _ in sched[2:])
+
+
+def test_kernel_work_counts_visible_pairs():
+    # a steady step of the bench layer: 32 heads x (1024 x 2048 + 1024 x 1025 / 2) pairs
+    pairs = bench.step_pairs(WL, WL.C, WL.T)
+    assert pairs == 32 * (1024 * 2048 + 1024 * 1025 // 2)
+    assert bench.kernel_work(WL, "sdpa_tc_kernel", WL.C, WL.T) == (4.0 * 128 * pairs, "flop", "tensor")
+    assert bench.kernel_work(WL, "wsum_tc_kernel", WL.C, WL.T)[0] == 2.0 * 128 * pairs
+
+
+def test_profiled_traffic_needs_matching_sources(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    csrc = root / "h2o_kv_cache_step_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("tc.cu", "tc_ptx.cuh", "common.cuh"):
+        shutil.copy(os.path.join(bench.ROOT, "h2o_kv_cache_step_b200", "csrc", f), csrc / f)
+    shutil.copy(os.path.join(bench.ROOT, "profiles", "dram_traffic.txt"), root / "profiles" / "dram_traffic.txt")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    sched = [(WL.C, WL.T)]  # the captured steady-state step itself: no scaling
+    rec = [l.split() for l in open(root / "profiles" / "dram_traffic.txt") if l.startswith("sdpa_tc_kernel")][0]
+    assert bench.profiled_traffic(WL, "sdpa_tc_kernel", sched) == pytest.approx(float(rec[4]) + float(rec[5]))
+    # launches that read less (a filling cache) are scaled by their compulsory bytes
+    small = bench.profiled_traffic(WL, "sdpa_tc_kernel", [(0, WL.T)])
+    assert small < float(rec[4])
+    # any change to the kernel's sources voids the record
+    with open(csrc / "tc.cu", "a") as fh:
+        fh.write("\n// changed\n")
+    assert bench.profiled_traffic(WL, "sdpa_tc_kernel", sched) is None
+    assert bench.profiled_traffic(WL, "scatter_kernel", sched) is None  # no record
+
+
+def test_job_throughput_is_all_ranks_over_the_slowest():
+    assert bench.job_throughput(65536, 4, 8.0) == pytest.approx(65536 * 4 / 0.008)
