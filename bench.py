@@ -110,11 +110,13 @@ def step_pairs(wl, n: int, T: int) -> int:
     return wl.B * wl.Hq * (T * n + T * (T + 1) // 2)
 
 
-def sequence_schedule(wl):
-    """(n before the step, T) for every chunk of one sequence prefill."""
+def sequence_schedule(wl, insert: bool = False):
+    """(cache entries the step attends to, T) for every chunk of one sequence
+    prefill: the n valid slots, or under insert-always the ones kept before
+    the attention (C - T once the chunk no longer fits)."""
     out, n = [], 0
     for _ in range(wl.n_chunks):
-        out.append((n, wl.T))
+        out.append((n if not insert or n + wl.T <= wl.C else wl.C - wl.T, wl.T))
         n = min(wl.C, n + wl.T)
     return out
 
@@ -211,7 +213,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     wl = rank_workload(synth.WORKLOADS[args.workload], rank, world)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    sched = sequence_schedule(wl)
+    sched = sequence_schedule(wl, insert=args.policy == "insert")
 
     t0 = time.time()
     chunks = []
@@ -224,9 +226,10 @@ def run_ours(args, rank, world, local_rank):
         f"in {time.time() - t0:.1f}s")
     out = torch.empty_like(chunks[0][0])
     cache = H2OCache(wl.B, wl.Hq, wl.Hkv, wl.d, wl.C, tdt, max_T=wl.T)
-    if args.policy == "normalized":
-        from h2o_kv_cache_step_b200._lib import H2O_POLICY_NORMALIZED
-        cache.set_policy(H2O_POLICY_NORMALIZED)
+    if args.policy != "sum":
+        from h2o_kv_cache_step_b200 import _lib
+        cache.set_policy({"normalized": _lib.H2O_POLICY_NORMALIZED,
+                          "insert": _lib.H2O_POLICY_INSERT_ALWAYS}[args.policy])
     plan = cache.kernel_plan(wl.T)
     stream = torch.cuda.current_stream()
 
@@ -242,7 +245,7 @@ def run_ours(args, rank, world, local_rank):
         st = tuple(torch.from_numpy(x).to(dev) for x in (K0, V0, S0, pos0))
         st = (st[0].to(tdt), st[1].to(tdt), st[2], st[3])
         c_idx = min(wl.n_chunks - 1, wl.C // wl.T + 1)
-        sched = [(wl.C, wl.T)]
+        sched = [(wl.C - wl.T if args.policy == "insert" else wl.C, wl.T)]
 
         def prefill():  # noqa: F811
             cache.set_state(*st, P=c_idx * wl.T, n=wl.C)
@@ -258,7 +261,7 @@ def run_ours(args, rank, world, local_rank):
         K0, V0, S0, pos0 = synth.random_state(wl, n=wl.C, P=P0, seed=1)
         st = tuple(torch.from_numpy(x).to(dev) for x in (K0, V0, S0, pos0))
         st = (st[0].to(tdt), st[1].to(tdt), st[2], st[3])
-        sched = [(wl.C, dT)] * D
+        sched = [(wl.C - dT if args.policy == "insert" else wl.C, dT)] * D
         dout = torch.empty_like(dchunks[0][0])
 
         def prefill():  # noqa: F811
@@ -511,8 +514,9 @@ def main():
                     help="prefill: a bench step is a whole-sequence prefill (default); chunk: one "
                          "steady-state chunk step (for profiler captures); decode: --decode-steps "
                          "steps of --decode-t tokens against a full cache")
-    ap.add_argument("--policy", default="sum", choices=["sum", "normalized"],
-                    help="eviction ranking: the H2O score (default) or score / age")
+    ap.add_argument("--policy", default="sum", choices=["sum", "normalized", "insert"],
+                    help="eviction: rank by the H2O score (default) or score / age, or insert-always "
+                         "(evict before the chunk attends)")
     ap.add_argument("--cpu-groups", type=int, default=0,
                     help="KV groups in the oracle sample (default: host cores)")
     args = ap.parse_args()

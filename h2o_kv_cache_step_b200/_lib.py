@@ -23,6 +23,7 @@ H2O_ERR_POISONED = -6
 H2O_ERR_UNSUPPORTED = -7
 H2O_POLICY_SUM = 0
 H2O_POLICY_NORMALIZED = 1
+H2O_POLICY_INSERT_ALWAYS = 2
 H2O_BF16 = 0
 H2O_FP32 = 1
 

@@ -58,6 +58,13 @@ struct h2o_ctx {
     size_t partial_elems = 0;
     float* nlse2 = nullptr;
     int rows_pad = 0;
+    // insert-always workspace (allocated when the policy is first selected):
+    // compact K/V of the kept entries, their slots, scores and positions
+    void* ins_K = nullptr;
+    void* ins_V = nullptr;
+    int32_t* ins_slot = nullptr;
+    float* ins_score = nullptr;
+    int32_t* ins_pos = nullptr;
     // decode-path workspace (chunks of up to kDecodeMaxT tokens)
     float* dec_part = nullptr;
     float* dec_logits = nullptr;
@@ -237,6 +244,11 @@ StepArgs make_args(h2o_ctx* c, const void* q, const void* k, const void* v, void
     a.partials = c->partials;
     a.partial_elems = c->partial_elems;
     a.nlse2 = c->nlse2;
+    a.ins_K = c->ins_K;
+    a.ins_V = c->ins_V;
+    a.ins_slot = c->ins_slot;
+    a.ins_score = c->ins_score;
+    a.ins_pos = c->ins_pos;
     a.dec_part = c->dec_part;
     a.dec_logits = c->dec_logits;
     a.dec_lse2 = c->dec_lse2;
@@ -327,6 +339,11 @@ int h2o_destroy(h2o_ctx* c) {
     for (cudaEvent_t e : c->prof_ev) cudaEventDestroy(e);
     cudaFree(c->Kc);
     cudaFree(c->Vc);
+    cudaFree(c->ins_K);
+    cudaFree(c->ins_V);
+    cudaFree(c->ins_slot);
+    cudaFree(c->ins_score);
+    cudaFree(c->ins_pos);
     cudaFree(c->scores);
     cudaFree(c->pos);
     cudaFree(c->stage);
@@ -355,17 +372,22 @@ int h2o_kernel_plan(const h2o_ctx* c, int T, const char** names, int max_names) 
     if (!c || T < 1) return fail(nullptr, H2O_ERR_ARG, "bad arguments");
     const char* plan[kMaxStepKernels];
     int k = 0;
+    const bool insert = c->policy == H2O_POLICY_INSERT_ALWAYS;
+    if (insert) {
+        plan[k++] = "insert_select_kernel";
+        plan[k++] = "gather_kernel";
+    }
     if (c->dec_part && decode_applies(c->Hq, c->Hkv, c->d, T)) {
         plan[k++] = "decode_split_kernel";
         plan[k++] = "decode_combine_kernel";
         plan[k++] = "decode_wsum_kernel";
     } else if (c->use_tc) {
-        k = tc_kernel_plan(c->B, c->Hq, c->Hkv, c->d, c->C, T, (int)c->n, plan, kMaxStepKernels - 2);
+        k += tc_kernel_plan(c->B, c->Hq, c->Hkv, c->d, c->C, T, (int)c->n, plan + k, kMaxStepKernels - 2 - k);
     } else {
         plan[k++] = "sdpa_simt_kernel";
         plan[k++] = "wsum_simt_kernel";
     }
-    plan[k++] = "select_kernel";
+    plan[k++] = insert ? "insert_finish_kernel" : "select_kernel";
     plan[k++] = "scatter_kernel";
     for (int i = 0; i < k && i < max_names; ++i)
         if (names) names[i] = plan[i];
@@ -380,6 +402,8 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
         return fail(c, H2O_ERR_ALIGN, "q, k, v, out must be 16-byte aligned");
     if (c->P + T > (int64_t)INT32_MAX) return fail(c, H2O_ERR_UNSUPPORTED, "positions would exceed 2^31-1");
+    if (c->policy == H2O_POLICY_INSERT_ALWAYS && T > c->C)
+        return fail(c, H2O_ERR_UNSUPPORTED, "insert-always needs T <= C (T = %d, C = %d)", T, c->C);
     DeviceGuard g(c->device);
     cudaStream_t s = (cudaStream_t)stream;
     if (T > c->tmax) {
@@ -401,19 +425,37 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
     }
     const bool decode = c->dec_part && decode_applies(c->Hq, c->Hkv, c->d, T);
     a.nparts = decode ? 1 : c->use_tc ? tc_partial_count(c->Hq, c->Hkv, T) : 0;
-    if (decode) {
-        H2O_TRY(c, launch_decode(a), "launch decode-path kernels");
-    } else if (c->use_tc) {
-        H2O_TRY(c, tc_sdpa(a), "launch tensor-core SDPA");
-        H2O_TRY(c, tc_wsum(a), "launch tensor-core weight sums");
-    } else {
-        H2O_TRY(c, launch_sdpa_simt(a), "launch SDPA");
-        H2O_TRY(c, launch_wsum_simt(a), "launch weight sums");
+    // insert-always: eviction first, then the chunk step over the compact
+    // cache of the kept entries (attention and weight sums unchanged)
+    const bool insert = c->policy == H2O_POLICY_INSERT_ALWAYS;
+    const int n_kept = insert ? (int)(c->n + T > c->C ? c->C - T : c->n) : (int)c->n;
+    StepArgs b = a;
+    if (insert) {
+        H2O_TRY(c, launch_insert_select(a, n_kept), "launch insert-always selection");
+        H2O_TRY(c, launch_gather(a, n_kept), "launch gather of the kept entries");
+        b.Kc = c->ins_K;
+        b.Vc = c->ins_V;
+        b.n = n_kept;
+        b.scores = c->ins_score;
+        b.pos = c->ins_pos;
     }
-    H2O_TRY(c, launch_select(a), "launch select");
+    if (decode) {
+        H2O_TRY(c, launch_decode(b), "launch decode-path kernels");
+    } else if (c->use_tc) {
+        H2O_TRY(c, tc_sdpa(b), "launch tensor-core SDPA");
+        H2O_TRY(c, tc_wsum(b), "launch tensor-core weight sums");
+    } else {
+        H2O_TRY(c, launch_sdpa_simt(b), "launch SDPA");
+        H2O_TRY(c, launch_wsum_simt(b), "launch weight sums");
+    }
+    if (insert) {
+        H2O_TRY(c, launch_insert_finish(a, n_kept), "launch insert-always score update");
+    } else {
+        H2O_TRY(c, launch_select(a), "launch select");
+    }
     H2O_TRY(c, launch_scatter(a), "launch scatter");
     c->last_T = T;
-    c->last_n = (int)c->n;
+    c->last_n = n_kept;  // the step's cache candidates (all n, or the kept ones under insert-always)
     c->n = std::min<int64_t>(c->C, c->n + T);
     c->P += T;
     return H2O_OK;
@@ -513,8 +555,18 @@ int h2o_step_host_async(h2o_ctx* c, const void* q, const void* k, const void* v,
 
 int h2o_set_policy(h2o_ctx* c, int policy) {
     if (!c) return fail(nullptr, H2O_ERR_ARG, "null context");
-    if (policy != H2O_POLICY_SUM && policy != H2O_POLICY_NORMALIZED)
+    if (policy != H2O_POLICY_SUM && policy != H2O_POLICY_NORMALIZED && policy != H2O_POLICY_INSERT_ALWAYS)
         return fail(c, H2O_ERR_ARG, "unknown eviction policy %d", policy);
+    if (policy == H2O_POLICY_INSERT_ALWAYS && !c->ins_K) {
+        DeviceGuard g(c->device);
+        const size_t groups = (size_t)c->B * c->Hkv;
+        const size_t rows = groups * c->C;
+        H2O_TRY(c, cudaMalloc(&c->ins_K, rows * c->d * c->elem), "cudaMalloc(compact K)");
+        H2O_TRY(c, cudaMalloc(&c->ins_V, rows * c->d * c->elem), "cudaMalloc(compact V)");
+        H2O_TRY(c, cudaMalloc(&c->ins_slot, sizeof(int32_t) * rows), "cudaMalloc(compact slots)");
+        H2O_TRY(c, cudaMalloc(&c->ins_score, sizeof(float) * rows), "cudaMalloc(compact scores)");
+        H2O_TRY(c, cudaMalloc(&c->ins_pos, sizeof(int32_t) * rows), "cudaMalloc(compact positions)");
+    }
     c->policy = policy;
     return H2O_OK;
 }

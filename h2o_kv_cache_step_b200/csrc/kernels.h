@@ -52,6 +52,11 @@ struct StepArgs {
     float* partials;     // weight-sum partials [nparts][B*Hkv][C+tmax] (tensor-core path)
     size_t partial_elems;
     int nparts;          // > 0: the selection kernel first sums the partials
+    void* ins_K;         // insert-always: compact K of the kept entries [B,Hkv,C,d]
+    void* ins_V;         // insert-always: compact V
+    int32_t* ins_slot;   // insert-always: slot of compact entry r [B*Hkv][C]
+    float* ins_score;    // insert-always: its score before the step
+    int32_t* ins_pos;    // insert-always: its position
     float* dec_part;     // decode path: per-(group, slice, row) partial O, max, sum
     float* dec_logits;   // decode path: scaled logits [group][row][C + kDecodeMaxT]
     float* dec_lse2;     // decode path: log2-sum-exp per (group, row)
@@ -129,6 +134,12 @@ size_t decode_part_floats(int B, int Hq, int Hkv, int d, int C);
 size_t decode_logit_floats(int B, int Hkv, int C);
 size_t decode_lse2_floats(int B, int Hkv);
 cudaError_t launch_decode(const StepArgs& a);
+
+// Insert-always variant: eviction before the attention, then the chunk step
+// over the compact cache of the kept entries.
+cudaError_t launch_insert_select(const StepArgs& a, int n_kept);
+cudaError_t launch_gather(const StepArgs& a, int n_kept);
+cudaError_t launch_insert_finish(const StepArgs& a, int n_kept);
 
 cudaError_t launch_select(const StepArgs& a);
 cudaError_t launch_scatter(const StepArgs& a);

@@ -80,8 +80,20 @@ enum h2o_dtype { H2O_BF16 = 0, H2O_FP32 = 1 };
  *                          with t = P + T the token count after the step and
  *                          t_j the candidate's position (every age >= 1).
  * Ties go to the larger position under both. The stored scores are phi
- * under both policies; only the ranking key differs. */
-enum h2o_policy { H2O_POLICY_SUM = 0, H2O_POLICY_NORMALIZED = 1 };
+ * under both policies; only the ranking key differs.
+ *   H2O_POLICY_INSERT_ALWAYS  the order the same section describes, new
+ *                          content overwriting the lowest-scoring slots:
+ *                          before the chunk attends, the n + T - C valid
+ *                          slots with the lowest scores so far are evicted
+ *                          (the older position first among equal scores);
+ *                          the T chunk tokens, in position order, take the
+ *                          empty and evicted slots in ascending order; then
+ *                          the rows attend to the buffer under the position
+ *                          mask of section "Kernel Support Needs" and every
+ *                          slot's score grows by its weights. Every chunk
+ *                          token enters, so a step needs T <= C
+ *                          (H2O_ERR_UNSUPPORTED otherwise). */
+enum h2o_policy { H2O_POLICY_SUM = 0, H2O_POLICY_NORMALIZED = 1, H2O_POLICY_INSERT_ALWAYS = 2 };
 
 /* Create a bf16 context on the current CUDA device: an empty cache of C slots
  * per (sequence, KV head), P = 0. Allocates all device memory it will need for
@@ -156,8 +168,10 @@ const char *h2o_last_error(const h2o_ctx *ctx);
  * is cache slot c, index n_prev + t is chunk token t, with n_prev the valid
  * slot count before that step. scores: updated score (old + weight sum);
  * pos: position; kept: 1 if it survived. Device arrays of [B, Hkv, ncand]
- * with ncand = n_prev + T_last (query it with h2o_last_step_info). Any of the
- * three pointers may be NULL. */
+ * with ncand = n_prev + T_last (query it with h2o_last_step_info). Under
+ * H2O_POLICY_INSERT_ALWAYS the cache candidates are the entries kept before
+ * the attention, in slot order (n_prev counts them), and every candidate is
+ * kept. Any of the three pointers may be NULL. */
 int h2o_candidates(h2o_ctx *ctx, float *scores, int32_t *pos, uint8_t *kept, void *stream);
 
 /* Slot each chunk token of the last step was written to, -1 if dropped:

@@ -83,6 +83,8 @@ def test_new_entry_points_reject_a_null_context(L):
 
 def test_policy_constants_match_the_header():
     src = open(os.path.join(ROOT, "include", "h2o.h")).read()
-    m = re.search(r"enum h2o_policy \{\s*H2O_POLICY_SUM = (\d+),\s*H2O_POLICY_NORMALIZED = (\d+)\s*\}", src)
+    m = re.search(r"enum h2o_policy \{\s*H2O_POLICY_SUM = (\d+),\s*H2O_POLICY_NORMALIZED = (\d+),"
+                  r"\s*H2O_POLICY_INSERT_ALWAYS = (\d+)\s*\}", src)
     assert m, "enum h2o_policy not found in h2o.h"
-    assert (int(m.group(1)), int(m.group(2))) == (_lib.H2O_POLICY_SUM, _lib.H2O_POLICY_NORMALIZED)
+    assert tuple(int(x) for x in m.groups()) == (_lib.H2O_POLICY_SUM, _lib.H2O_POLICY_NORMALIZED,
+                                                 _lib.H2O_POLICY_INSERT_ALWAYS)

@@ -94,6 +94,51 @@ def test_normalized_policy_lockstep(dtype, d, B, Hq, Hkv, C, T, chunks):
     assert differs
 
 
+@pytest.mark.parametrize("dtype,d,B,Hq,Hkv,C,T,chunks,full", [
+    ("bf16", 128, 2, 8, 2, 256, 96, 5, False),   # fills, then evicts before attending (tensor cores)
+    ("bf16", 128, 1, 8, 2, 200, 200, 3, False),  # T = C: the whole cache turns over every step
+    ("fp32", 64, 1, 4, 2, 130, 33, 6, False),    # CUDA-core path
+    ("bf16", 128, 1, 8, 2, 300, 4, 4, True),     # short chunks on a full cache: decode path
+])
+def test_insert_always_lockstep(dtype, d, B, Hq, Hkv, C, T, chunks, full):
+    """H2O_POLICY_INSERT_ALWAYS against the oracle's insert-always step from
+    the device's own state each step: outputs and LSE within tolerance, token
+    slots and positions exact, scores within tolerance, the chunk's rows in
+    their slots."""
+    from h2o_kv_cache_step_b200._lib import H2O_POLICY_INSERT_ALWAYS
+    wl = synth.Workload("insert", dtype, B=B, Hq=Hq, Hkv=Hkv, d=d, C=C, T=T, N=T * chunks, seed=17,
+                        recipe="heavy", hh_frac=0.05)
+    cache = H2OCache(B, Hq, Hkv, d, C, TORCH_DTYPE[dtype], max_T=T)
+    cache.set_policy(H2O_POLICY_INSERT_ALWAYS)
+    if full:
+        K, V, S, pos = synth.random_state(wl, n=C, P=2000, seed=3)
+        cache.set_state(to_dev(K, dtype), to_dev(V, dtype), torch.from_numpy(S).cuda(),
+                        torch.from_numpy(pos).cuda(), P=2000, n=C)
+    for c in range(chunks):
+        q, k, v = synth.chunk(wl, c)
+        pre = oracle_state_from_device(cache)
+        st = pre.copy()
+        out_ref, lse_ref, ts_ref = oracle.step_insert_always(st, q, k, v)
+        g = gpu_step(cache, q, k, v, dtype)
+        assert np.abs(g["out"] - out_ref).max() <= TOL_OUT[dtype]
+        assert np.abs(g["lse"] - lse_ref).max() <= TOL_LSE[dtype]
+        assert np.array_equal(g["token_slot"], ts_ref)
+        assert np.array_equal(g["Pos"], st.pos.astype(np.int32))
+        compare_scores(g["S"], st.phi, "insert-always scores")
+        for b in range(B):
+            for gg in range(Hkv):
+                assert np.array_equal(g["K"][b, gg, ts_ref[b, gg]], np.asarray(k, np.float32)[b, gg])
+
+
+def test_insert_always_rejects_chunks_longer_than_the_cache():
+    from h2o_kv_cache_step_b200._lib import H2O_POLICY_INSERT_ALWAYS, H2OError
+    cache = H2OCache(1, 2, 1, 64, 8, torch.float32, max_T=16)
+    cache.set_policy(H2O_POLICY_INSERT_ALWAYS)
+    x = torch.zeros((1, 2, 9, 64), device="cuda")
+    with pytest.raises(H2OError):
+        cache.step(x, x[:, :1].contiguous(), x[:, :1].contiguous())
+
+
 def test_set_policy_rejects_unknown():
     from h2o_kv_cache_step_b200._lib import H2OError
     cache = H2OCache(1, 2, 1, 64, 8, torch.float32, max_T=4)
