@@ -22,6 +22,8 @@
  *      with the largest score survive (equal scores: the larger position
  *      survives); kept cache entries stay in their slots, and the kept chunk
  *      tokens, in position order, fill the free slots in ascending slot order.
+ * That is the default policy; h2o_set_policy selects the normalized ranking
+ * or the insert-always order instead (enum h2o_policy).
  *
  * Conventions for every entry point:
  *   - Every call returns a status (H2O_OK or a negative H2O_ERR_*); none
@@ -109,13 +111,17 @@ int h2o_create_ex(int B, int Hq, int Hkv, int d, int C, int dtype, int max_T, h2
  * NULL is accepted. */
 int h2o_destroy(h2o_ctx *ctx);
 
+/* Select the eviction policy (enum h2o_policy) for the following steps; the
+ * default is H2O_POLICY_SUM. Takes effect from the next h2o_step; call it
+ * between steps (it is not stream-ordered). The first selection of
+ * H2O_POLICY_INSERT_ALWAYS allocates that variant's workspace (a compact copy
+ * of the cache and per-slot arrays; H2O_ERR_CUDA / H2O_ERR_OOM if that
+ * fails). H2O_ERR_ARG for an unknown policy. */
+int h2o_set_policy(h2o_ctx *ctx, int policy);
+
 /* One H2O step on the chunk (q, k, v) of T tokens (device pointers, layouts
  * above); writes the attention output to out (device). Updates the cache,
  * scores and positions; P advances by T. Asynchronous on `stream`. */
-/* Select the eviction ranking (enum h2o_policy) for the following steps.
- * Takes effect from the next h2o_step; H2O_ERR_ARG for an unknown policy. */
-int h2o_set_policy(h2o_ctx *ctx, int policy);
-
 int h2o_step(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
              int T, void *stream);
 
