@@ -37,25 +37,29 @@ def build(force: bool = False) -> str:
     return _SO
 
 
+def bind(L):
+    """Declare the oracle's C signatures on a loaded library; returns it."""
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    L.h2o_oracle_step.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 15 + [I]
+    L.h2o_oracle_step.restype = I
+    L.h2o_oracle_step_policy.argtypes = [I, I, I, I, I, I, ctypes.c_int64, I] + [P] * 15 + [I]
+    L.h2o_oracle_step_policy.restype = I
+    L.h2o_oracle_step_insert.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 10 + [I]
+    L.h2o_oracle_step_insert.restype = I
+    L.h2o_oracle_backward.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 12 + [I]
+    L.h2o_oracle_backward.restype = I
+    L.h2o_oracle_select_group.argtypes = [I, I, I, P, P, P, P, P]
+    L.h2o_oracle_select_group.restype = I
+    L.h2o_oracle_rows.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 6 + [I, P, P, P, I]
+    L.h2o_oracle_rows.restype = I
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        L.h2o_oracle_step.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 15 + [I]
-        L.h2o_oracle_step.restype = I
-        L.h2o_oracle_step_policy.argtypes = [I, I, I, I, I, I, ctypes.c_int64, I] + [P] * 15 + [I]
-        L.h2o_oracle_step_policy.restype = I
-        L.h2o_oracle_step_insert.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 10 + [I]
-        L.h2o_oracle_step_insert.restype = I
-        L.h2o_oracle_backward.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 12 + [I]
-        L.h2o_oracle_backward.restype = I
-        L.h2o_oracle_select_group.argtypes = [I, I, I, P, P, P, P, P]
-        L.h2o_oracle_select_group.restype = I
-        L.h2o_oracle_rows.argtypes = [I, I, I, I, I, I, ctypes.c_int64] + [P] * 6 + [I, P, P, P, I]
-        L.h2o_oracle_rows.restype = I
-        _lib = L
+        _lib = bind(ctypes.CDLL(build()))
     return _lib
 
 
