@@ -32,12 +32,32 @@ MUTANTS = {
 }
 
 
+# mistakes in the normalized policy, the insert-always variant and the backward
+MUTANTS.update({
+    "normalized: age off by one": ("cand_score[c] / (double)(t_after - cand_pos[c])",
+                                   "cand_score[c] / (double)(t_after - cand_pos[c] + 1)"),
+    "insert-always: the highest evicted": (
+        "if (b != a && pos[b] >= 0 && ranks_above(phi[a], pos[a], phi[b], pos[b])) ++below;",
+        "if (b != a && pos[b] >= 0 && ranks_above(phi[b], pos[b], phi[a], pos[a])) ++below;"),
+    "insert-always: chunk token hidden from its own row": (
+        "if (pos[j] < 0 || pos[j] > P + i) continue;\n                w[j] =",
+        "if (pos[j] < 0 || pos[j] > P + i || (pos[j] == P + i && i > 0)) continue;\n                w[j] ="),
+    "backward: row-sum term dropped": ("const double ds = p[j] * (dp[j] - pdp);", "const double ds = p[j] * dp[j];"),
+    "backward: dV without the weights": ("gv[x] += p[j] * go[x];", "gv[x] += go[x];"),
+})
+
+
 def _battery():
     """Pins that together should fail for any of the mistakes above."""
     pins.test_hand_worked_example(None, "worked_example_c2_t2.json")
+    pins.test_hand_worked_example(None, "worked_example_c2_t2_normalized.json")
     pins.test_oracle_matches_brute_force(None, 2, 4, 2, 8, 6, 3, 5, 1.0, False)
     pins.test_oracle_matches_brute_force(None, 1, 2, 1, 5, 4, 1, 9, 2.0, False)
+    pins.test_oracle_matches_brute_force(None, 2, 4, 2, 8, 6, 3, 5, 1.0, True)
     pins.test_select_against_sort_with_planted_ties(None, 0)
+    pins.test_insert_always_hand_worked_example(None)
+    pins.test_insert_always_matches_brute_force(None, 2, 4, 2, 8, 6, 3, 5, 1.0)
+    pins.test_backward_matches_torch_autograd(None)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
