@@ -44,6 +44,10 @@ MUTANTS.update({
         "if (pos[j] < 0 || pos[j] > P + i || (pos[j] == P + i && i > 0)) continue;\n                w[j] ="),
     "backward: row-sum term dropped": ("const double ds = p[j] * (dp[j] - pdp);", "const double ds = p[j] * dp[j];"),
     "backward: dV without the weights": ("gv[x] += p[j] * go[x];", "gv[x] += go[x];"),
+    # the per-row checker used at full size
+    "rows: a row does not see its own token": ("const int n_keys = C + i + 1;", "const int n_keys = C + i;"),
+    "rows: KV head of the wrong group": ("const size_t bg = (size_t)b * Hkv + g;\n        const double *qrow",
+                                         "const size_t bg = (size_t)b * Hkv + h % Hkv;\n        const double *qrow"),
 })
 
 
@@ -58,6 +62,7 @@ def _battery():
     pins.test_insert_always_hand_worked_example(None)
     pins.test_insert_always_matches_brute_force(None, 2, 4, 2, 8, 6, 3, 5, 1.0)
     pins.test_backward_matches_torch_autograd(None)
+    pins.test_rows_match_brute_force(None, 2, 4, 2, 8, 9, 4, 5)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -441,3 +441,67 @@ def test_backward_equal_values_give_no_query_or_key_gradient(oracle_lib):
     for g in range(k.shape[1]):
         total = dVc[0, g].sum(axis=0) + dv[0, g].sum(axis=0)
         np.testing.assert_allclose(total, dout[0, g * G:(g + 1) * G].sum(axis=(0, 1)), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------ selected rows -----
+def _all_rows(B, Hq, T):
+    return np.array([(b, h, i) for b in range(B) for h in range(Hq) for i in range(T)], np.int32)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,C,T,n_chunks", [
+    (2, 4, 2, 8, 9, 4, 5),     # GQA; cache partly empty (n < C) in the first steps, then evicting
+    (1, 6, 2, 5, 7, 5, 4),     # G = 3, T = 5 (ragged against any tile)
+    (1, 2, 2, 4, 3, 7, 3),     # chunk longer than the cache
+    (1, 4, 1, 6, 5, 1, 8),     # T = 1: only row 0, which is also row T - 1
+])
+def test_rows_match_brute_force(oracle_lib, B, Hq, Hkv, d, C, T, n_chunks):
+    """The per-row checker (O and LSE of chosen rows against the pre-step
+    cache) agrees with the structurally different brute force on every row of
+    every step: a cold cache, a partly filled one and a full one."""
+    gen = iid_gen(B, Hq, Hkv, d, T, seed=C * 31 + T)
+    st = oracle.State.empty(B, Hkv, C, d)
+    br = brute.BruteH2O(B, Hq, Hkv, d, C)
+    rows = _all_rows(B, Hq, T)
+    saw_partial = saw_full = False
+    for c in range(n_chunks):
+        q, k, v = gen(c)
+        n_before = st.n_valid
+        saw_partial |= bool(((n_before > 0) & (n_before < C)).any())
+        saw_full |= bool((n_before == C).all())
+        o_rows, l_rows = oracle.rows(st, q, k, v, rows)
+        bo, bl, _, _ = br.step(q, k, v)
+        oracle.step(st, q, k, v)
+        for r, (b, h, i) in enumerate(rows):
+            np.testing.assert_allclose(o_rows[r], bo[b, h, i], rtol=0, atol=1e-12)
+            assert abs(l_rows[r] - bl[b, h, i]) <= 1e-12
+    assert saw_full and (saw_partial or C <= T)
+
+
+def test_rows_match_dense_causal_attention(oracle_lib):
+    """With no eviction, row i of chunk c is row c*T + i of full causal
+    attention (textbook softmax attention over the whole prefix)."""
+    B, Hq, Hkv, d, T, n_chunks = 1, 4, 2, 8, 6, 4
+    N = T * n_chunks
+    r = np.random.default_rng(12)
+    qa = r.standard_normal((B, Hq, N, d))
+    ka = r.standard_normal((B, Hkv, N, d))
+    va = r.standard_normal((B, Hkv, N, d))
+    dout, dlse, _ = brute.dense_causal(qa, ka, va)
+    st = oracle.State.empty(B, Hkv, N + 2, d)
+    # rows 0 and T - 1 of every head, plus one interior row
+    rows = np.array([(0, h, i) for h in range(Hq) for i in (0, 2, T - 1)], np.int32)
+    for c in range(n_chunks):
+        sl = slice(c * T, c * T + T)
+        o_rows, l_rows = oracle.rows(st, qa[:, :, sl], ka[:, :, sl], va[:, :, sl], rows)
+        for j, (b, h, i) in enumerate(rows):
+            np.testing.assert_allclose(o_rows[j], dout[b, h, c * T + i], rtol=0, atol=1e-12)
+            assert abs(l_rows[j] - dlse[b, h, c * T + i]) <= 1e-12
+        oracle.step(st, qa[:, :, sl], ka[:, :, sl], va[:, :, sl])
+
+
+def test_rows_rejects_out_of_range_rows(oracle_lib):
+    st = oracle.State.empty(1, 1, 4, 2)
+    q, k, v = iid_gen(1, 2, 1, 2, 3, seed=1)(0)
+    for bad in ((1, 0, 0), (0, 2, 0), (0, 0, 3), (0, -1, 0)):
+        with pytest.raises(RuntimeError):
+            oracle.rows(st, q, k, v, np.array([bad], np.int32))
