@@ -558,14 +558,29 @@ int h2o_set_policy(h2o_ctx* c, int policy) {
     if (policy != H2O_POLICY_SUM && policy != H2O_POLICY_NORMALIZED && policy != H2O_POLICY_INSERT_ALWAYS)
         return fail(c, H2O_ERR_ARG, "unknown eviction policy %d", policy);
     if (policy == H2O_POLICY_INSERT_ALWAYS && !c->ins_K) {
+        // all five buffers or none: a failed allocation leaves the context as
+        // it was (policy unchanged, no buffer recorded), so a retry starts over
         DeviceGuard g(c->device);
         const size_t groups = (size_t)c->B * c->Hkv;
         const size_t rows = groups * c->C;
-        H2O_TRY(c, cudaMalloc(&c->ins_K, rows * c->d * c->elem), "cudaMalloc(compact K)");
-        H2O_TRY(c, cudaMalloc(&c->ins_V, rows * c->d * c->elem), "cudaMalloc(compact V)");
-        H2O_TRY(c, cudaMalloc(&c->ins_slot, sizeof(int32_t) * rows), "cudaMalloc(compact slots)");
-        H2O_TRY(c, cudaMalloc(&c->ins_score, sizeof(float) * rows), "cudaMalloc(compact scores)");
-        H2O_TRY(c, cudaMalloc(&c->ins_pos, sizeof(int32_t) * rows), "cudaMalloc(compact positions)");
+        void* bufs[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+        const size_t bytes[5] = {rows * c->d * c->elem, rows * c->d * c->elem, sizeof(int32_t) * rows,
+                                 sizeof(float) * rows, sizeof(int32_t) * rows};
+        for (int i = 0; i < 5; ++i) {
+            const cudaError_t e = cudaMalloc(&bufs[i], bytes[i]);
+            if (e != cudaSuccess) {
+                for (int j = 0; j < i; ++j) cudaFree(bufs[j]);
+                cudaGetLastError();  // an allocation failure is not sticky: clear it
+                return fail(c, e == cudaErrorMemoryAllocation ? H2O_ERR_OOM : H2O_ERR_CUDA,
+                            "cudaMalloc of the insert-always workspace (%zu bytes): %s", bytes[i],
+                            cudaGetErrorString(e));
+            }
+        }
+        c->ins_K = bufs[0];
+        c->ins_V = bufs[1];
+        c->ins_slot = static_cast<int32_t*>(bufs[2]);
+        c->ins_score = static_cast<float*>(bufs[3]);
+        c->ins_pos = static_cast<int32_t*>(bufs[4]);
     }
     c->policy = policy;
     return H2O_OK;

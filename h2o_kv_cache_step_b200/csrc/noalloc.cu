@@ -13,6 +13,7 @@
 // The scratch array is a file-scope __device__ object: every GPU that loads
 // the library holds it (kNoAllocScratchInts int32, 1 MiB) until the process
 // exits, whether or not the entry point is ever called.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -33,9 +34,30 @@ constexpr int kThreads = 1024;
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 
 // Device address of g_noalloc_scratch per device (host code cannot use the
-// symbol itself as a device pointer).
+// symbol itself as a device pointer), with the CUDA context it was looked up
+// in: after a device reset the library's module is loaded again in a new
+// context, possibly at another address, so a changed context means a new
+// lookup.
 int32_t* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 std::mutex g_scratch_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, fetched through the runtime (the library
+// does not link the driver API); nullptr if unavailable.
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
+}
 
 
 __device__ __forceinline__ uint32_t na_ordered_bits(float s) {
@@ -191,19 +213,25 @@ int na_fail(int code, const char* msg) {
 }
 
 // Device address of the scratch array on the current device; looked up once
-// per device (the first call on a device does it).
+// per device and context (the first call on a device does it, and the first
+// call after the device's context changed, e.g. after cudaDeviceReset).
 int scratch_address(int32_t** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return na_fail(H2O_ERR_CUDA, "h2o_select_noalloc: cudaGetDevice failed");
     if (dev < 0 || dev >= kMaxDevices) return na_fail(H2O_ERR_UNSUPPORTED, "h2o_select_noalloc: device index too large");
+    CtxGetCurrentFn get = ctx_get_current_fn();
+    CUcontext ctx = nullptr;
+    if (get && get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (g_scratch_addr[dev] == nullptr || ctx == nullptr || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // also makes the context current
         if (e != cudaSuccess || p == nullptr)
             return na_fail(H2O_ERR_CUDA, "h2o_select_noalloc: cudaGetSymbolAddress of the scratch array failed");
+        if (get && get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
         g_scratch_addr[dev] = static_cast<int32_t*>(p);
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_addr[dev];
     return H2O_OK;

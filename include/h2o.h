@@ -116,7 +116,8 @@ int h2o_destroy(h2o_ctx *ctx);
  * between steps (it is not stream-ordered). The first selection of
  * H2O_POLICY_INSERT_ALWAYS allocates that variant's workspace (a compact copy
  * of the cache and per-slot arrays; H2O_ERR_CUDA / H2O_ERR_OOM if that
- * fails). H2O_ERR_ARG for an unknown policy. */
+ * fails, in which case nothing stays allocated and the policy is unchanged).
+ * H2O_ERR_ARG for an unknown policy. */
 int h2o_set_policy(h2o_ctx *ctx, int policy);
 
 /* One H2O step on the chunk (q, k, v) of T tokens (device pointers, layouts
@@ -247,8 +248,9 @@ int h2o_profile_end(h2o_ctx *ctx, int max_kernels, const char **names, double *t
  * buffer. Scratch (the free-slot lists) lives in a static device array of
  * 262144 int32 (1 MiB) that every GPU loading the library holds until exit;
  * groups * C above that returns H2O_ERR_UNSUPPORTED. The first call on a
- * device looks up that array's device address (once per device); make that
- * first call before any stream capture. Each device has its own copy of the
+ * device looks up that array's device address (once per device, and again
+ * when the device's CUDA context has changed, as after cudaDeviceReset); make
+ * that first call before any stream capture. Each device has its own copy of the
  * array and every call on that device shares it, keeping whatever the last
  * call left there: calls that overlap on the GPU (for example on two streams)
  * race, so serialise them. Nothing in it needs clearing between calls. Asynchronous on `stream`; errors are

@@ -10,7 +10,7 @@ import torch
 from h2o_kv_cache_step_b200 import H2OCache, synth
 from oracle import oracle
 from parity_util import (TOL_LSE, TOL_OUT, TORCH_DTYPE, check_selection_replay, compare_scores,
-                         gpu_step, lockstep_full, oracle_state_from_device, to_dev)
+                         gpu_step, lockstep_full, oracle_state_from_device, record_errors, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -185,6 +185,29 @@ def test_decode_path_limits():
     assert cache2.kernel_plan(17)[0] == "sdpa_simt_kernel"
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_selection_fallback_for_large_candidate_sets(dtype):
+    """Candidate sets whose 64-bit keys do not fit in shared memory (C + T =
+    32,832 here) take the selection kernel's other form, which rebuilds each
+    key from the candidate arrays on every radix pass. Two evicting steps
+    from a full cache, lockstep against the oracle with the selection replayed
+    bit-exactly."""
+    C, T = 32768, 64
+    m = C + T
+    smem_limit = 220 * 1024  # the selection kernel's shared-memory budget
+    assert m * 8 + m + 4 * C > smem_limit >= m + 4 * C  # keys do not fit; flags and free list do
+    wl = synth.Workload("select-fallback", dtype, B=1, Hq=2, Hkv=1, d=64, C=C, T=T, N=2 * T, seed=23,
+                        recipe="heavy", hh_frac=0.05)
+    cache = H2OCache(wl.B, wl.Hq, wl.Hkv, wl.d, C, TORCH_DTYPE[dtype], max_T=T)
+    K, V, S, pos = synth.random_state(wl, n=C, P=100000, seed=5)
+    cache.set_state(to_dev(K, dtype), to_dev(V, dtype), torch.from_numpy(S).cuda(),
+                    torch.from_numpy(pos).cuda(), P=100000, n=C)
+    for c in range(2):
+        q, k, v = synth.chunk(wl, c)
+        lockstep_full(cache, q, k, v, dtype, C)
+
+
 def test_cache_of_one_slot():
     wl = synth.Workload("c1slot", "fp32", B=1, Hq=2, Hkv=1, d=64, C=1, T=5, N=20, seed=2)
     run_sequence_lockstep(wl)
@@ -329,6 +352,7 @@ def test_full_size_sampled(name, policy):
     o_ref, l_ref = oracle.rows(pre, q, k, v, rows)
     o_gpu = g["out"][rows[:, 0], rows[:, 1], rows[:, 2]]
     l_gpu = g["lse"][rows[:, 0], rows[:, 1], rows[:, 2]]
+    record_errors(f"full size {name} sampled rows", o_gpu, o_ref, l_gpu, l_ref)
     assert np.abs(o_gpu - o_ref).max() <= TOL_OUT["bf16"]
     assert np.abs(l_gpu - l_ref).max() <= TOL_LSE["bf16"]
     # one whole group through the full oracle step

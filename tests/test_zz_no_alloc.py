@@ -7,7 +7,9 @@ where an allocation would synchronise the device): it keeps its scratch in a
 static device array instead of a context-owned buffer. Fed the candidate
 scores and positions a real step produced, it must reproduce that step's
 kept flags, token slots, slot scores and slot positions exactly (selection
-is integer/bit-exact work), on two steps in a row. This file is collected
+is integer/bit-exact work), on two steps in a row; the oracle's selection on
+the same candidates must agree, and a call must leave the device's free
+memory unchanged. This file is collected
 last so that a failure here cannot hide any other test."""
 import ctypes
 
@@ -26,6 +28,7 @@ def _p(t):
 def test_select_noalloc_matches_step_eviction():
     from h2o_kv_cache_step_b200 import H2OCache, synth
     from h2o_kv_cache_step_b200._lib import H2O_ERR_UNSUPPORTED, H2O_OK, lib
+    from oracle import oracle
 
     wl = synth.Workload("noalloc", "bf16", B=2, Hq=8, Hkv=2, d=128, C=192, T=128, N=128 * 4,
                         seed=21, recipe="heavy", hh_frac=0.04)
@@ -50,15 +53,38 @@ def test_select_noalloc_matches_step_eviction():
         ps = pos_before.clone()
         kept = torch.full_like(kept_step, 7)
         ts = torch.full_like(slots_step, -9)
+        # outputs of a second call, allocated before it
+        sc2, ps2 = scores_before.clone(), pos_before.clone()
+        kept2, ts2 = torch.full_like(kept_step, 5), torch.full_like(slots_step, -5)
+        stream = torch.cuda.current_stream()
+        calls += 1
         rc = lib().h2o_select_noalloc(groups, wl.C, n, wl.T, P, _p(cand_s), _p(cand_p), _p(sc), _p(ps),
-                                      _p(kept), _p(ts), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+                                      _p(kept), _p(ts), ctypes.c_void_p(stream.cuda_stream))
         assert rc == H2O_OK, lib().h2o_last_error(None)
         torch.cuda.synchronize()
+        if calls == 1:
+            # after the first call on the device, a call leaves the device's
+            # free memory exactly as it was: it allocates nothing
+            free_before = torch.cuda.mem_get_info()[0]
+            rc = lib().h2o_select_noalloc(groups, wl.C, n, wl.T, P, _p(cand_s), _p(cand_p), _p(sc2), _p(ps2),
+                                          _p(kept2), _p(ts2), ctypes.c_void_p(stream.cuda_stream))
+            assert rc == H2O_OK, lib().h2o_last_error(None)
+            torch.cuda.synchronize()
+            assert torch.cuda.mem_get_info()[0] == free_before
+            # the replayed call computed the same result
+            assert torch.equal(kept2, kept) and torch.equal(ts2, ts)
+            # and the oracle's selection on the same candidates agrees
+            for grp in range(groups):
+                slot = np.concatenate([np.arange(n, dtype=np.int32), np.full(wl.T, -1, np.int32)])
+                kept_ref, ts_ref = oracle.select_group(
+                    wl.C, wl.T, cand_s.reshape(groups, -1)[grp].double().cpu().numpy(),
+                    cand_p.reshape(groups, -1)[grp].long().cpu().numpy(), slot)
+                assert np.array_equal(kept_ref, kept.reshape(groups, -1)[grp].cpu().numpy())
+                assert np.array_equal(ts_ref, ts.reshape(groups, -1)[grp].cpu().numpy())
         assert torch.equal(kept, kept_step)
         assert torch.equal(ts, slots_step)
         assert torch.equal(ps, pos_step)
         assert torch.equal(sc.view(torch.int32), scores_step.view(torch.int32))
-        calls += 1
     assert calls >= 2  # two evicting steps in a row
 
     # sizes beyond the built-in scratch are refused, with a message
