@@ -15,10 +15,12 @@
 // (matrix row) per thread.
 //
 // SDPA: M = 128 query rows, N = 128 keys per block, K = d; two query tiles
-//   (two heads of one KV group) per CTA, 11 warps: Q/K loader, MMA issuer,
-//   two softmax warpgroups, V loader. S = Q K^T lands in the tile's TMEM
-//   buffer; its softmax warpgroup turns it into P (bf16, written to shared
-//   memory in the 128-byte-swizzled K-major layout the next MMA reads) and
+//   (two heads of one KV group) per CTA, 11 warps: a loader (Q, and K / V
+//   through a three-slot ring), one MMA-issuing warp per tile, and one softmax
+//   warpgroup per tile. S = Q K^T lands in the tile's TMEM buffer; its softmax
+//   warpgroup reads the row in one pass (S is then free for the next QK),
+//   turns it into P (bf16, written to shared memory in the 128-byte-swizzled
+//   K-major layout the next MMA reads, in two halves of 64 keys) and
 //   O += P V accumulates in TMEM. The running maximum is only moved (and O
 //   rescaled in TMEM) when it grows by more than 2^16, so most blocks skip the
 //   rescale. One pair of exponentials in every four goes through a degree-3
@@ -95,38 +97,43 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // One CTA per SM works on two query tiles at once: rows m0..m0+127 of query
 // heads hA and hB = hA + 1 of the same KV group, so both see the same keys and
 // every K/V block is loaded once for the pair. TMEM (512 columns) holds S and O
-// (128 + d columns) per tile. Each tile has its own softmax warpgroup, which
-// loads S(j) into registers and releases its TMEM columns at once, so QK(j+1)
-// runs on the tensor core while the softmax of block j is still computing;
-// P goes to shared memory (128-byte-swizzled, K-major) for the PV MMA. The
-// tile's serial chain is therefore only its softmax; the tensor core sees
-// QK and PV of both tiles interleaved.
+// (128 + d columns) per tile.
+//
+// Per key block j and tile X, the tile's softmax warpgroup reads the whole S
+// row (128 fp32 values) into registers in one pass and releases S at once, so
+// QK(j+1) runs on the tensor core while the exponentials of block j are
+// computed. P goes to shared memory (bf16, 128-byte-swizzled, K-major) in two
+// halves of 64 keys, each with its own full / consumed barriers: the PV MMA of
+// the first half starts while the second half is computed, and the softmax of
+// block j+1 only waits for the half of PV(j) whose buffer it overwrites.
+// K and V blocks share a ring of three shared-memory slots, loaded in the
+// order K0, K1, V0, K2, V1, ... so that each K block arrives a whole block
+// before the QK that needs it.
 // A group with an odd number of query heads leaves one single-tile CTA per
 // (group, row tile).
 template <int D>
 struct SdpaCfg {
     static constexpr int HALF = 128 * 128;       // bytes of one 128-row x 64-col bf16 box
     static constexpr int TILE = 128 * D * 2;     // one 128-row x d tile
-    static constexpr int PB = 128 * 128 * 2;     // one P tile (128 rows x 128 keys, bf16)
-    static constexpr int KS = 2;                 // K stages (V has one buffer)
+    static constexpr int PB = 2 * HALF;          // one P tile (128 rows x 128 keys, bf16), two halves
+    static constexpr int RING = 3;               // K/V slots
     static constexpr int OFF_QA = 0;
     static constexpr int OFF_QB = TILE;
-    static constexpr int OFF_K = 2 * TILE;
-    static constexpr int OFF_V = OFF_K + KS * TILE;
-    static constexpr int OFF_P = OFF_V + TILE;   // [2 tiles]
+    static constexpr int OFF_RING = 2 * TILE;
+    static constexpr int OFF_P = OFF_RING + RING * TILE;  // [2 tiles]
     static constexpr int OFF_BAR = OFF_P + 2 * PB;
     static constexpr int NBAR = 24;
     static constexpr int SMEM_RAW = OFF_BAR + NBAR * 8 + 16 + 1024;
     // more than half of an SM's shared memory, so one CTA (512 TMEM columns) per SM
     static constexpr int SMEM = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
     static constexpr uint32_t TMEM_COLS = 512;
-    // warp 0 loads Q and K, warp 1 issues the MMAs, warps 2..9 are the two
-    // softmax warpgroups, warp 10 loads V. The two loaders need warps of their
-    // own: a lane that sleeps in an mbarrier wait suspends its whole warp.
+    // warp 0 loads Q, K and V, warps 2..9 are the two softmax warpgroups,
+    // warps 1 and 10 issue the MMAs of tiles A and B
     static constexpr int THREADS = 352;
     static constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, D, true);
 };
+static_assert(SdpaCfg<128>::SMEM_RAW <= 232448, "SDPA shared memory exceeds the per-CTA limit");
 
 struct SdpaParams {
     int B, Hq, Hkv, T, C, n, tmax;
@@ -147,20 +154,18 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                const __grid_constant__ CUtensorMap map_vc, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const SdpaParams p) {
     using Cfg = SdpaCfg<D>;
-    constexpr int KS = Cfg::KS;
+    constexpr int RING = Cfg::RING;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;           // [KS]
-    uint64_t* k_empty = k_full + KS;       // [KS]
-    uint64_t* v_full = k_empty + KS;
-    uint64_t* v_empty = v_full + 1;
-    uint64_t* s_full = v_empty + 1;        // [2 tiles]
-    uint64_t* s_free = s_full + 2;         // [2 tiles], 4 arrivals: S loaded into registers
-    uint64_t* p_full = s_free + 2;         // [2 tiles], 4 arrivals: P written to shared memory
-    uint64_t* pv_done = p_full + 2;        // [2 tiles]
-    uint64_t* drain = pv_done + 2;
+    uint64_t* ring_full = bars + 1;            // [RING]
+    uint64_t* ring_empty = ring_full + RING;   // [RING]
+    uint64_t* s_full = ring_empty + RING;      // [2 tiles]
+    uint64_t* s_free = s_full + 2;             // [2 tiles], 4 arrivals: S loaded into registers
+    uint64_t* p_full = s_free + 2;             // [2 tiles][2 halves], 4 arrivals: P half in shared memory
+    uint64_t* pv_done = p_full + 4;            // [2 tiles][2 halves]: PV of that half completed
+    uint64_t* drain = pv_done + 4;             // [2 tiles]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -179,19 +184,20 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < KS; ++s) {
-            mbar_init(k_full + s, 1);
-            mbar_init(k_empty + s, 1);
+        for (int s = 0; s < RING; ++s) {
+            mbar_init(ring_full + s, 1);
+            mbar_init(ring_empty + s, hasB ? 2 : 1);  // released by each tile's MMA warp
         }
-        mbar_init(v_full, 1);
-        mbar_init(v_empty, 1);
         for (int t = 0; t < 2; ++t) {
             mbar_init(s_full + t, 1);
             mbar_init(s_free + t, 4);
-            mbar_init(p_full + t, 4);
-            mbar_init(pv_done + t, 1);
+            for (int h = 0; h < 2; ++h) {
+                mbar_init(p_full + 2 * t + h, 4);
+                mbar_init(pv_done + 2 * t + h, 1);
+            }
         }
         mbar_init(drain, 1);
+        mbar_init(drain + 1, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -204,14 +210,16 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     griddep_wait();  // inputs written, and the previous step's readers done
     griddep_launch_dependents();
 
-    if (warp == 0 || warp == 10) {
-        // ---------------------------------------------------------- producers
-        // warp 0: Q and the K ring; warp 10: the V buffer
-        if (warp == 0 && lane == 0) {
+    if (warp == 0) {
+        // ----------------------------------------------------------- producer
+        // Q of both tiles, then K0, K1, V0, K2, V1, ..., K(nb-1), V(nb-2), V(nb-1)
+        // through the ring
+        if (lane == 0) {
             tc::prefetch_tmap(&map_q);
             tc::prefetch_tmap(&map_kc);
+            tc::prefetch_tmap(&map_vc);
             tc::prefetch_tmap(&map_k);
-            int kcount[KS] = {};
+            tc::prefetch_tmap(&map_v);
             mbar_arrive_expect_tx(q_full, Cfg::TILE * (hasB ? 2 : 1));
             for (int hh = 0; hh < D / 64; ++hh) {
                 tc::tma_load_2d(smem + Cfg::OFF_QA + hh * Cfg::HALF, &map_q, 64 * hh, (b * p.Hq + hA) * p.T + m0,
@@ -220,124 +228,115 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     tc::tma_load_2d(smem + Cfg::OFF_QB + hh * Cfg::HALF, &map_q, 64 * hh,
                                     (b * p.Hq + hA + 1) * p.T + m0, q_full);
             }
-            for (int j = 0; j < nb; ++j) {
+            int L = 0;
+            auto load_kv = [&](bool isV, int j) -> bool {
+                const int slot = L % RING;
+                if (!wait_bar(ring_empty + slot, ((L / RING) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag))
+                    return false;
                 const bool cache = j < p.nbc;
                 const int row = cache ? bg * p.C + 128 * j : bg * p.T + 128 * (j - p.nbc);
-                const int ks = j % KS;
-                if (!wait_bar(k_empty + ks, ((j / KS) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(k_full + ks, Cfg::TILE);
+                const CUtensorMap* map = isV ? (cache ? &map_vc : &map_v) : (cache ? &map_kc : &map_k);
+                mbar_arrive_expect_tx(ring_full + slot, Cfg::TILE);
                 for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_K + ks * Cfg::TILE + hh * Cfg::HALF, cache ? &map_kc : &map_k,
-                                    64 * hh, row, k_full + ks);
-                ++kcount[ks];
+                    tc::tma_load_2d(smem + Cfg::OFF_RING + slot * Cfg::TILE + hh * Cfg::HALF, map, 64 * hh, row,
+                                    ring_full + slot);
+                ++L;
+                return true;
+            };
+            bool ok = load_kv(false, 0);
+            for (int j = 0; ok && j < nb; ++j) {
+                if (j + 1 < nb) ok = load_kv(false, j + 1);
+                if (ok) ok = load_kv(true, j);
             }
+            // every load issued here has landed before the CTA may exit
             wait_bar(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
-            for (int s = 0; s < KS; ++s)
-                if (kcount[s]) wait_bar(k_full + s, (kcount[s] - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-        } else if (warp == 10 && lane == 0) {
-            tc::prefetch_tmap(&map_vc);
-            tc::prefetch_tmap(&map_v);
-            int vcount = 0;
-            for (int j = 0; j < nb; ++j) {
-                const bool cache = j < p.nbc;
-                const int row = cache ? bg * p.C + 128 * j : bg * p.T + 128 * (j - p.nbc);
-                if (!wait_bar(v_empty, (j & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)) break;
-                mbar_arrive_expect_tx(v_full, Cfg::TILE);
-                for (int hh = 0; hh < D / 64; ++hh)
-                    tc::tma_load_2d(smem + Cfg::OFF_V + hh * Cfg::HALF, cache ? &map_vc : &map_v, 64 * hh, row,
-                                    v_full);
-                ++vcount;
+            for (int s = 0; s < RING; ++s) {
+                const int uses = L / RING + (s < L % RING ? 1 : 0);
+                if (uses) wait_bar(ring_full + s, (uses - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
             }
-            if (vcount) wait_bar(v_full, (vcount - 1) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
         }
-    } else if (warp == 1) {
-        // ----------------------------------------------------------- MMA issuer
-        const uint32_t sQA = sbase + Cfg::OFF_QA, sQB = sbase + Cfg::OFF_QB, sV = sbase + Cfg::OFF_V;
-        const uint32_t tSA = tmem, tOA = tmem + 128, tSB = tmem + 256, tOB = tmem + 384;
-        auto issue_qk = [&](uint32_t dS, uint32_t sQ, int ks) {
-            const uint32_t sK = sbase + Cfg::OFF_K + ks * Cfg::TILE;
+    } else if (warp == 1 || (warp == 10 && hasB)) {
+        // ---------------------------------------------------------- MMA issuers
+        // one warp per tile (warp 1: tile A, warp 10: tile B), so that the
+        // waits and issue overhead of one tile overlap the other's; the
+        // tensor core takes both streams. Every descriptor is a base value
+        // plus a constant offset (the start-address field is the byte
+        // address / 16 in the low bits, and no address here reaches 2^18).
+        const int X = warp == 1 ? 0 : 1;
+        const uint32_t tS = tmem + 256 * X, tO = tmem + 256 * X + 128;
+        const uint64_t dQ = desc_kmajor_sw128(sbase + (X ? Cfg::OFF_QB : Cfg::OFF_QA));
+        const uint64_t dRingK = desc_kmajor_sw128(sbase + Cfg::OFF_RING);
+        const uint64_t dRingV = desc_mnmajor_sw128(sbase + Cfg::OFF_RING, Cfg::HALF);
+        const uint64_t dP = desc_kmajor_sw128(sbase + Cfg::OFF_P + X * Cfg::PB);
+        auto issue_qk = [&](int slot) {
+            const uint64_t dK = dRingK + (uint64_t)((slot * Cfg::TILE) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-                tc::mma_bf16_ss(dS, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(sK + off), Cfg::IDESC_QK, kk > 0);
+                const uint32_t off = ((kk >> 2) * Cfg::HALF + (kk & 3) * 32) >> 4;
+                tc::mma_bf16_ss(tS, dQ + off, dK + off, Cfg::IDESC_QK, kk > 0);
             }
         };
-        auto issue_pv = [&](uint32_t dO, int tile, bool first) {
-            const uint32_t sP = sbase + Cfg::OFF_P + tile * Cfg::PB;
+        // O += P[:, 64h .. 64h+63] V[64h .. 64h+63, :]
+        auto issue_pv_half = [&](int slot, int h, bool first) {
+            const uint64_t dV = dRingV + (uint64_t)((slot * Cfg::TILE) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per instruction
-                const uint32_t aoff = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-                tc::mma_bf16_ss(dO, desc_kmajor_sw128(sP + aoff), desc_mnmajor_sw128(sV + kk * 16 * 128, Cfg::HALF),
-                                Cfg::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < 4; ++k4) {  // 64 keys, 16 per instruction
+                const int kk = 4 * h + k4;
+                tc::mma_bf16_ss(tO, dP + (uint64_t)((h * Cfg::HALF + k4 * 32) >> 4),
+                                dV + (uint64_t)((kk * 16 * 128) >> 4), Cfg::IDESC_PV, (!first || k4 > 0) ? 1u : 0u);
             }
         };
-        bool ok = warp_wait(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag) &&
-                  warp_wait(k_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag);
+        int L = 0;
+        auto wait_ring = [&](int& slot) -> bool {
+            slot = L % RING;
+            const bool r = warp_wait(ring_full + slot, (L / RING) & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
+            ++L;
+            return r;
+        };
+        int ks = 0;
+        bool ok = warp_wait(q_full, 0, p.wb, kDevTimeoutTmaWait, abort_flag) && wait_ring(ks);
         if (ok) {
-            fence_after_sync();
             if (lane == 0) {
-                issue_qk(tSA, sQA, 0);
-                tc::mma_commit(s_full);
-                if (hasB) {
-                    issue_qk(tSB, sQB, 0);
-                    tc::mma_commit(s_full + 1);
-                }
-                tc::mma_commit(k_empty);
+                issue_qk(ks);
+                tc::mma_commit(s_full + X);
+                tc::mma_commit(ring_empty + ks);
             }
             __syncwarp();
         }
         for (int j = 0; ok && j < nb; ++j) {
-            // QK(., j + 1) as soon as each softmax has taken S(j) out of TMEM
+            // QK(j + 1) as soon as the softmax has taken S(j) out of TMEM
             if (j + 1 < nb) {
-                const int ks = (j + 1) % KS;
-                ok = warp_wait(k_full + ks, ((j + 1) / KS) & 1, p.wb, kDevTimeoutTmaWait, abort_flag) &&
-                     warp_wait(s_free, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                ok = wait_ring(ks) && warp_wait(s_free + X, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
                 if (!ok) break;
                 fence_after_sync();
                 if (lane == 0) {
-                    issue_qk(tSA, sQA, ks);
-                    tc::mma_commit(s_full);
+                    issue_qk(ks);
+                    tc::mma_commit(s_full + X);
+                    tc::mma_commit(ring_empty + ks);
                 }
                 __syncwarp();
-                if (hasB) {
-                    if (!(ok = warp_wait(s_free + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag))) break;
-                    fence_after_sync();
-                    if (lane == 0) {
-                        issue_qk(tSB, sQB, ks);
-                        tc::mma_commit(s_full + 1);
-                    }
-                    __syncwarp();
-                }
-                if (lane == 0) tc::mma_commit(k_empty + ks);
-                __syncwarp();
             }
-            // PV(., j) once P(j) is in shared memory
-            ok = warp_wait(p_full, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag) &&
-                 warp_wait(v_full, j & 1, p.wb, kDevTimeoutTmaWait, abort_flag);
-            if (!ok) break;
-            fence_after_sync();
-            if (lane == 0) {
-                issue_pv(tOA, 0, j == 0);
-                tc::mma_commit(pv_done);
-            }
-            __syncwarp();
-            if (hasB) {
-                if (!(ok = warp_wait(p_full + 1, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag))) break;
+            // PV(j) half by half, as the softmax hands P over
+            int vs = 0;
+            if (!(ok = wait_ring(vs))) break;
+            for (int h = 0; h < 2; ++h) {
+                if (!(ok = warp_wait(p_full + 2 * X + h, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag))) break;
                 fence_after_sync();
                 if (lane == 0) {
-                    issue_pv(tOB, 1, j == 0);
-                    tc::mma_commit(pv_done + 1);
+                    issue_pv_half(vs, h, j == 0 && h == 0);
+                    tc::mma_commit(pv_done + 2 * X + h);
                 }
                 __syncwarp();
             }
-            if (lane == 0) tc::mma_commit(v_empty);
+            if (!ok) break;
+            if (lane == 0) tc::mma_commit(ring_empty + vs);
             __syncwarp();
         }
         // all MMAs issued here complete before TMEM can be released
-        if (lane == 0) tc::mma_commit(drain);
+        if (lane == 0) tc::mma_commit(drain + X);
         __syncwarp();
-        warp_wait(drain, 0, p.wb, kDevTimeoutMmaWait, abort_flag);
-    } else if (warp < 6 || hasB) {
+        warp_wait(drain + X, 0, p.wb, kDevTimeoutMmaWait, abort_flag);
+    } else if (warp >= 2 && warp < 10 && (warp < 6 || hasB)) {
         // -------------------------------------------------------------- softmax
         const int X = warp < 6 ? 0 : 1;     // which tile
         const int h = hA + X;
@@ -347,135 +346,128 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int r = quad * 32 + lane;  // row inside the tile = TMEM lane
         const int i = m0 + r;            // query row inside the chunk
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        uint8_t* prow = prow_base + r * 128;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
             ok = warp_wait(s_full + X, j & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
             if (!ok) break;
             fence_after_sync();
+            // the whole row of S in one pass; S is free for QK(j+1) right after
+            uint32_t v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tS + lane_off + 32 * c, v[c]);
+            tc::tmem_ld_wait();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free + X);
             // visible columns of this row in block j: col < limit
             const int limit = (j < p.nbc) ? p.n - 128 * j : min(i, p.T - 1) - 128 * (j - p.nbc) + 1;
-            // pass 1 (TMEM): maximum of the raw visible scores (the scale is positive)
+            if (limit < 128) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * c + e >= limit) v[c][e] = __float_as_uint(-INFINITY);
+            }
+            // row maximum of the raw scores (the scale is positive)
             float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                uint32_t v[2][32];
-                tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
-                tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
-                tc::tmem_ld_wait();
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    const int cbase = 64 * c2 + 32 * hv;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float a0 = (cbase + e < limit) ? __uint_as_float(v[hv][e]) : -INFINITY;
-                        const float a1 = (cbase + e + 1 < limit) ? __uint_as_float(v[hv][e + 1]) : -INFINITY;
-                        if ((e >> 1) & 1) mx1 = tc::max3(mx1, a0, a1);
-                        else mx0 = tc::max3(mx0, a0, a1);
-                    }
+                for (int e = 0; e < 32; e += 4) {
+                    mx0 = tc::max3(mx0, __uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1]));
+                    mx1 = tc::max3(mx1, __uint_as_float(v[c][e + 2]), __uint_as_float(v[c][e + 3]));
                 }
-            }
             // the running maximum only moves when it grows by more than 2^16
             const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * p.scale_log2);
             const bool resc = m_new > m_run + kRescaleThreshold;
             const float m_use = resc ? m_new : m_run;
             const float alpha = resc ? ex2(m_run - m_use) : 1.f;
-            // PV(j-1) has completed: the P buffer is free and O is stable
-            if (j > 0) {
-                ok = warp_wait(pv_done + X, (j - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
-                if (__any_sync(0xffffffffu, resc)) {
+            // P = 2^(s * scale - m) -> bf16 -> shared memory, one half of the
+            // keys at a time
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 nm2 = make_float2(-m_use, -m_use);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t v[32];
-                        tc::tmem_ld32(tO + lane_off + 32 * c, v);
-                        tc::tmem_ld_wait();
+            for (int hf = 0; hf < 2; ++hf) {
+                // the half's buffer is free once PV(j-1) of the same half has
+                // completed (after a give-up the stores are harmless: nothing
+                // reads them)
+                if (j > 0 && ok) ok = warp_wait(pv_done + 2 * X + hf, (j - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                        tc::tmem_st32(tO + lane_off + 32 * c, v);
-                    }
-                    tc::tmem_st_wait();
-                }
-            }
-            // pass 2 (TMEM): P = 2^(s * scale - m) -> bf16 -> shared memory; S is
-            // released after its last load so that QK(j+1) can start
-            const float nm = -m_use;
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            uint8_t* prow = prow_base + r * 128;
+                for (int cc = 0; cc < 8; ++cc) {  // 8 keys (16 bytes of P) at a time
+                    const int c = 2 * hf + (cc >> 2);
+                    const int e0 = 8 * (cc & 3);
+                    uint32_t pk[4];
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                uint32_t v[2][32];
-                tc::tmem_ld32(tS + lane_off + 64 * c2, v[0]);
-                tc::tmem_ld32(tS + lane_off + 64 * c2 + 32, v[1]);
-                tc::tmem_ld_wait();
-                if (c2 == 1) {
-                    fence_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(s_free + X);
-                }
-#pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-#pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        const int col = 64 * c2 + 32 * hv + 8 * c8;
-                        float e[8];
-#pragma unroll
-                        for (int k = 0; k < 8; k += 2) {
-                            const float x0 = fmaf(__uint_as_float(v[hv][8 * c8 + k]), p.scale_log2, nm);
-                            const float x1 = fmaf(__uint_as_float(v[hv][8 * c8 + k + 1]), p.scale_log2, nm);
-                            if ((k >> 1) < kPolyPairsOf4Sdpa) {
-                                const float2 pe = tc::exp2_poly3_x2_ftz(make_float2(x0, x1));
-                                e[k] = pe.x;
-                                e[k + 1] = pe.y;
-                            } else {
-                                e[k] = ex2(x0);
-                                e[k + 1] = ex2(x1);
-                            }
+                    for (int k = 0; k < 8; k += 2) {
+                        const float2 x = tc::ffma2(
+                            make_float2(__uint_as_float(v[c][e0 + k]), __uint_as_float(v[c][e0 + k + 1])), sc2, nm2);
+                        float2 pe;
+                        if ((k >> 1) < kPolyPairsOf4Sdpa) {
+                            pe = tc::exp2_poly3_x2_ftz(x);
+                        } else {
+                            pe.x = ex2(x.x);
+                            pe.y = ex2(x.y);
                         }
                         if (limit < 128) {
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) e[k] = (col + k < limit) ? e[k] : 0.f;
+                            const int col = 32 * c + e0 + k;
+                            pe.x = col < limit ? pe.x : 0.f;
+                            pe.y = col + 1 < limit ? pe.y : 0.f;
                         }
-                        s0 = tc::fadd_ftz(s0, e[0] + e[4]);
-                        s1 = tc::fadd_ftz(s1, e[1] + e[5]);
-                        s2 = tc::fadd_ftz(s2, e[2] + e[6]);
-                        s3 = tc::fadd_ftz(s3, e[3] + e[7]);
-                        uint4 val;
-                        val.x = tc::pack_bf16(e[0], e[1]);
-                        val.y = tc::pack_bf16(e[2], e[3]);
-                        val.z = tc::pack_bf16(e[4], e[5]);
-                        val.w = tc::pack_bf16(e[6], e[7]);
-                        const int ch = col >> 3, half = ch >> 3, cc = ch & 7;
-                        *reinterpret_cast<uint4*>(prow + half * Cfg::HALF + ((cc ^ (r & 7)) << 4)) = val;
+                        if ((k >> 1) & 1) acc1 = tc::fadd2_ftz(acc1, pe);
+                        else acc0 = tc::fadd2_ftz(acc0, pe);
+                        pk[k >> 1] = tc::pack_bf16(pe.x, pe.y);
+                    }
+                    *reinterpret_cast<uint4*>(prow + hf * Cfg::HALF + ((cc ^ (r & 7)) << 4)) =
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+                if (hf == 0 && j > 0 && ok && __any_sync(0xffffffffu, resc)) {
+                    // rescale O once PV(j-1) has completed (its last half implies
+                    // both), before PV(j) accumulates into it
+                    ok = warp_wait(pv_done + 2 * X + 1, (j - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag);
+                    if (ok) {
+                        fence_after_sync();
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tc::tmem_ld32(tO + lane_off + 32 * c, o);
+                            tc::tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tc::tmem_st32(tO + lane_off + 32 * c, o);
+                        }
+                        tc::tmem_st_wait();
                     }
                 }
+                tc::fence_proxy_async_smem();
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full + 2 * X + hf);
             }
-            tc::fence_proxy_async_smem();
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + X);
-            l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
+            if (!ok) break;
+            l_run = l_run * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
             m_run = m_use;
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && warp_wait(pv_done + X, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
+        if (ok && warp_wait(pv_done + 2 * X + 1, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
             fence_after_sync();
             const float inv = 1.f / l_run;
             __nv_bfloat16* orow = p.out + ((size_t)(b * p.Hq + h) * p.T + i) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                tc::tmem_ld32(tO + lane_off + 32 * c, v);
+                uint32_t o[32];
+                tc::tmem_ld32(tO + lane_off + 32 * c, o);
                 tc::tmem_ld_wait();
                 if (i < p.T) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         uint4 val;
-                        val.x = tc::pack_bf16(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
-                        val.y = tc::pack_bf16(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
-                        val.z = tc::pack_bf16(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
-                        val.w = tc::pack_bf16(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
+                        val.x = tc::pack_bf16(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+                        val.y = tc::pack_bf16(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+                        val.z = tc::pack_bf16(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+                        val.w = tc::pack_bf16(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
                         *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q4) = val;
                     }
                 }
