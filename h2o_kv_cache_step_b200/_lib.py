@@ -41,6 +41,7 @@ SIGNATURES = [
     ("h2o_destroy", _I, [_P]),
     ("h2o_step", _I, [_P, _P, _P, _P, _P, _I, _P]),
     ("h2o_step_host", _I, [_P, _P, _P, _P, _P, _I, _P]),
+    ("h2o_backward", _I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
     ("h2o_step_host_async", _I, [_P, _P, _P, _P, _P, _I, _P]),
     ("h2o_host_sync", _I, [_P]),
     ("h2o_set_policy", _I, [_P, _I]),

@@ -76,6 +76,32 @@ class H2OCache:
                                    _stream_ptr(stream)))
         return out
 
+    def backward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lse: torch.Tensor,
+                 dout: torch.Tensor, stream=None):
+        """Gradients of one step's attention for the key set it used, taking the
+        cache as it stands now as that step's pre-step cache (restore it with
+        set_state first when replaying). lse is the step's log-sum-exp.
+        Returns fp32 (dq, dK, dV, dk, dv): dK, dV over the cache slots
+        [B,Hkv,C,d], dk, dv over the chunk [B,Hkv,T,d]."""
+        T = q.shape[2]
+        for name, t, heads in (("q", q, self.Hq), ("k", k, self.Hkv), ("v", v, self.Hkv),
+                               ("dout", dout, self.Hq)):
+            if (t.dtype != self.dtype or not t.is_cuda or not t.is_contiguous()
+                    or tuple(t.shape) != (self.B, heads, T, self.d)):
+                raise ValueError(f"{name}: need contiguous CUDA {self.dtype} of shape "
+                                 f"{(self.B, heads, T, self.d)}, got {t.dtype} {tuple(t.shape)}")
+        if lse.dtype != torch.float32 or tuple(lse.shape) != (self.B, self.Hq, T) or not lse.is_contiguous():
+            raise ValueError("lse: need contiguous float32 [B, Hq, T]")
+        f32 = dict(dtype=torch.float32, device=self.device)
+        dq = torch.empty((self.B, self.Hq, T, self.d), **f32)
+        dK = torch.empty((self.B, self.Hkv, self.C, self.d), **f32)
+        dV = torch.empty_like(dK)
+        dk = torch.empty((self.B, self.Hkv, T, self.d), **f32)
+        dv = torch.empty_like(dk)
+        self._check(lib().h2o_backward(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(dout), T,
+                                       _ptr(dq), _ptr(dK), _ptr(dV), _ptr(dk), _ptr(dv), _stream_ptr(stream)))
+        return dq, dK, dV, dk, dv
+
     def set_policy(self, policy: int) -> None:
         """Eviction ranking for the following steps: _lib.H2O_POLICY_SUM (the
         H2O score, default) or _lib.H2O_POLICY_NORMALIZED (score / age)."""

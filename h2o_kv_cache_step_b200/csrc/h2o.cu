@@ -65,6 +65,10 @@ struct h2o_ctx {
     int32_t* ins_slot = nullptr;
     float* ins_score = nullptr;
     int32_t* ins_pos = nullptr;
+    // backward workspace (allocated on the first h2o_backward): dO . O and the
+    // log2-domain LSE per flattened group row, [2][groups][bwd_rows_pad]
+    float* bwd_rows = nullptr;
+    int bwd_rows_pad = 0;
     // decode-path workspace (chunks of up to kDecodeMaxT tokens)
     float* dec_part = nullptr;
     float* dec_logits = nullptr;
@@ -339,6 +343,7 @@ int h2o_destroy(h2o_ctx* c) {
     for (cudaEvent_t e : c->prof_ev) cudaEventDestroy(e);
     cudaFree(c->Kc);
     cudaFree(c->Vc);
+    cudaFree(c->bwd_rows);
     cudaFree(c->ins_K);
     cudaFree(c->ins_V);
     cudaFree(c->ins_slot);
@@ -458,6 +463,73 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
     c->last_n = n_kept;  // the step's cache candidates (all n, or the kept ones under insert-always)
     c->n = std::min<int64_t>(c->C, c->n + T);
     c->P += T;
+    return H2O_OK;
+}
+
+int h2o_backward(h2o_ctx* c, const void* q, const void* k, const void* v, const float* lse, const void* dout,
+                 int T, float* dq, float* dK, float* dV, float* dk, float* dv, void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (T < 1) return fail(c, H2O_ERR_ARG, "T must be >= 1 (got %d)", T);
+    if (!q || !k || !v || !lse || !dout || !dq || !dK || !dV || !dk || !dv)
+        return fail(c, H2O_ERR_ARG, "every pointer argument must be non-NULL");
+    for (const void* p : {q, k, v, dout, (const void*)lse, (const void*)dq, (const void*)dK, (const void*)dV,
+                          (const void*)dk, (const void*)dv})
+        if (!aligned16(p)) return fail(c, H2O_ERR_ALIGN, "every pointer argument must be 16-byte aligned");
+    DeviceGuard g(c->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int rows_pad = tc_rows_pad(c->Hq, c->Hkv, T);
+    if (rows_pad > c->bwd_rows_pad) {
+        // first use, or a longer chunk than before: (re)allocate once
+        if (c->bwd_rows) {
+            H2O_TRY(c, cudaStreamSynchronize(s), "sync before backward workspace growth");
+            H2O_TRY(c, cudaDeviceSynchronize(), "sync before backward workspace growth");
+            cudaFree(c->bwd_rows);
+            c->bwd_rows = nullptr;
+            c->bwd_rows_pad = 0;
+        }
+        H2O_TRY(c, cudaMalloc(&c->bwd_rows, sizeof(float) * 2 * (size_t)c->B * c->Hkv * rows_pad),
+                "cudaMalloc(backward row tables)");
+        c->bwd_rows_pad = rows_pad;
+    }
+    BwdArgs a{};
+    a.B = c->B;
+    a.Hq = c->Hq;
+    a.Hkv = c->Hkv;
+    a.d = c->d;
+    a.C = c->C;
+    a.T = T;
+    a.n = (int)c->n;
+    a.dtype = c->dtype;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.lse = lse;
+    a.dout = dout;
+    a.Kc = c->Kc;
+    a.Vc = c->Vc;
+    a.dq = dq;
+    a.dKc = dK;
+    a.dVc = dV;
+    a.dk = dk;
+    a.dv = dv;
+    a.rows_pad = c->bwd_rows_pad;
+    a.Drow = c->bwd_rows;
+    a.L2row = c->bwd_rows + (size_t)c->B * c->Hkv * c->bwd_rows_pad;
+    a.wb.err_word = c->err_dev;
+    a.wb.ns = c->wait_ns;
+    a.stream = s;
+    a.num_sms = c->num_sms;
+    LaunchLog local_log;
+    a.log = &local_log;
+    if (c->prof_on && c->prof_steps < c->prof_max_steps) {
+        const int slot = c->prof_steps++;
+        a.log = &c->prof_logs[slot];
+        a.log->n = 0;
+        a.log->ev = &c->prof_ev[(size_t)slot * (kMaxStepKernels + 1)];
+        H2O_TRY(c, cudaEventRecord(a.log->ev[0], s), "record profiling event");
+    }
+    H2O_TRY(c, launch_bwd_simt(a), "launch backward");
     return H2O_OK;
 }
 

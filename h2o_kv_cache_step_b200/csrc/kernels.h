@@ -141,6 +141,34 @@ cudaError_t launch_insert_select(const StepArgs& a, int n_kept);
 cudaError_t launch_gather(const StepArgs& a, int n_kept);
 cudaError_t launch_insert_finish(const StepArgs& a, int n_kept);
 
+// Backward of one step's chunk SDPA with the key set held fixed (the replay of
+// a logged step): everything the kernels read or write. Device pointers.
+struct BwdArgs {
+    int B, Hq, Hkv, d, C, T;
+    int n;              // valid cache slots (prefix 0..n-1) of the replayed pre-step cache
+    int dtype;          // 0 = bf16, 1 = fp32 (inputs); gradients are fp32
+    const void* q;      // [B,Hq,T,d]
+    const void* k;      // [B,Hkv,T,d]
+    const void* v;      // [B,Hkv,T,d]
+    const float* lse;   // forward natural-log LSE [B,Hq,T]
+    const void* dout;   // dL/dout [B,Hq,T,d]
+    const void* Kc;     // [B,Hkv,C,d]
+    const void* Vc;     // [B,Hkv,C,d]
+    float* dq;          // [B,Hq,T,d]
+    float* dKc;         // [B,Hkv,C,d] (zero in empty slots)
+    float* dVc;         // [B,Hkv,C,d]
+    float* dk;          // [B,Hkv,T,d]
+    float* dv;          // [B,Hkv,T,d]
+    float* Drow;        // [B*Hkv][rows_pad]: sum_j p_j dp_j / sum_j p_j per flattened group row (head-in-group * T + i)
+    float* L2row;       // [B*Hkv][rows_pad]: log2-domain LSE per flattened group row
+    int rows_pad;
+    WaitBound wb;
+    cudaStream_t stream;
+    int num_sms;
+    LaunchLog* log;
+};
+cudaError_t launch_bwd_simt(const BwdArgs& a);
+
 cudaError_t launch_select(const StepArgs& a);
 cudaError_t launch_scatter(const StepArgs& a);
 // Sets the message h2o_last_error(NULL) reports on this thread.

@@ -126,6 +126,28 @@ int h2o_set_policy(h2o_ctx *ctx, int policy);
 int h2o_step(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
              int T, void *stream);
 
+/* Backward of one step's chunk SDPA with the step's key set held fixed
+ * ("Learning how to Forget", paper page, section "Gradient Computation
+ * Strategy for Sparse Attention": training through the sparse cache replays
+ * the logged eviction decisions, so each step's attention is differentiated
+ * for the keys it actually attended to; the eviction carries no gradient).
+ * The context's current cache (K, V and the n valid slots, as h2o_set_state
+ * left it) is taken as the step's pre-step cache and is not modified; q, k,
+ * v are the step's chunk (device, layouts above, context dtype), lse its
+ * natural-log LSE (device float [B, Hq, T], as h2o_lse returned after the
+ * step) and dout = dL/dout [B, Hq, T, d] (context dtype). Writes, as device
+ * float (fp32) arrays,
+ *   dq [B, Hq, T, d], dK, dV [B, Hkv, C, d] (the cache slots; zero in empty
+ *   slots), dk, dv [B, Hkv, T, d] (the chunk),
+ * with the key / value gradients of a KV head summed over the query heads of
+ * its group. The row term sum_j p_j dp_j (= dout . out) is recomputed from
+ * the attention weights, so the step's output is not an input. Every pointer
+ * must be 16-byte aligned. The first call (and one with a longer chunk than
+ * before) allocates the backward's row workspace. Asynchronous on `stream`. */
+int h2o_backward(h2o_ctx *ctx, const void *q, const void *k, const void *v, const float *lse,
+                 const void *dout, int T, float *dq, float *dK, float *dV, float *dk, float *dv,
+                 void *stream);
+
 /* h2o_step with HOST buffers: copies q, k, v to library-owned device staging
  * buffers, runs the step and copies the output back into out (host). Page-
  * locked host memory gives asynchronous copies; pageable memory works too.
