@@ -21,9 +21,9 @@
 // factor near 1 instead of a term e * D_i * sum_j p_j k_j. dq_i then comes out
 // of one pass over the keys as scale * (sum_j p_j dp_j k_j - D_i sum_j p_j k_j).
 //
-// These kernels take every dtype and head dimension the library supports and
-// compute in fp32; the tensor-core kernels (backward_tc.cu) take the bf16
-// inputs of the sm_100a path.
+// These kernels carry the fp32 path (and any context without the tensor-core
+// path) and compute in fp32; backward_tc.cu holds the tcgen05 kernels of the
+// bf16 path.
 #include "kernels.h"
 
 namespace h2o {

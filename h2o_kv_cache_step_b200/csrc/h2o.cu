@@ -529,7 +529,11 @@ int h2o_backward(h2o_ctx* c, const void* q, const void* k, const void* v, const 
         a.log->ev = &c->prof_ev[(size_t)slot * (kMaxStepKernels + 1)];
         H2O_TRY(c, cudaEventRecord(a.log->ev[0], s), "record profiling event");
     }
-    H2O_TRY(c, launch_bwd_simt(a), "launch backward");
+    if (c->use_tc) {
+        H2O_TRY(c, tc_backward(a), "launch tensor-core backward");
+    } else {
+        H2O_TRY(c, launch_bwd_simt(a), "launch backward");
+    }
     return H2O_OK;
 }
 

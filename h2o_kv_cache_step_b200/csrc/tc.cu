@@ -61,36 +61,6 @@ constexpr float kRescaleThreshold = 16.f;  // log2 units
 constexpr int kPolyPairsOf4Sdpa = H2O_POLY_SDPA;  // SDPA: pairs in every 4 on the FMA pipe
 constexpr int kPolyPairsOf8Wsum = H2O_POLY_WSUM;  // weight sums: pairs in every 8 on the FMA pipe
 
-// Bounded wait that also gives up once another role has given up.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitBound& wb, int code,
-                                         volatile int* abort_flag) {
-    const uint32_t addr = smem_u32(bar);
-    if (mbar_try_wait(addr, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    while (true) {
-        for (int i = 0; i < 8; ++i)
-            if (mbar_try_wait_sleep(addr, parity, 20000u)) return true;
-        if (*abort_flag) return false;
-        if (global_ns() - t0 > wb.ns) {
-            record_error(wb, code);
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
-
-// Every lane waits; the outcome is made warp-uniform so that a give-up never
-// leaves part of a warp behind at a warp-collective instruction.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitBound& wb, int code,
-                                          volatile int* abort_flag) {
-    return __all_sync(0xffffffffu, wait_bar(bar, parity, wb, code, abort_flag));
-}
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    const uint32_t a = smem_u32(p);
-    return p + (((a + 1023u) & ~1023u) - a);
-}
-
 // ============================================================================
 // SDPA
 // ============================================================================
@@ -825,7 +795,7 @@ EncodeTiledFn encode_fn() {
 
 // 2-D map over a [rows, d] bf16 matrix, boxes of box_rows rows x 64 columns,
 // 128-byte swizzle (the layout the UMMA descriptors above describe).
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows = 128) {
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
@@ -844,9 +814,11 @@ cudaError_t sdpa_launch(const StepArgs& a) {
     using Cfg = SdpaCfg<D>;
     if (cudaError_t e = ensure_smem_limit(sdpa_tc_kernel<D>, Cfg::SMEM); e != cudaSuccess) return e;
     CUtensorMap mq, mkc, mvc, mk, mv;
-    if (!make_map(&mq, a.q, (uint64_t)a.B * a.Hq * a.T, D) || !make_map(&mkc, a.Kc, (uint64_t)a.B * a.Hkv * a.C, D) ||
-        !make_map(&mvc, a.Vc, (uint64_t)a.B * a.Hkv * a.C, D) || !make_map(&mk, a.k, (uint64_t)a.B * a.Hkv * a.T, D) ||
-        !make_map(&mv, a.v, (uint64_t)a.B * a.Hkv * a.T, D))
+    if (!make_map(&mq, a.q, (uint64_t)a.B * a.Hq * a.T, D, 128) ||
+        !make_map(&mkc, a.Kc, (uint64_t)a.B * a.Hkv * a.C, D, 128) ||
+        !make_map(&mvc, a.Vc, (uint64_t)a.B * a.Hkv * a.C, D, 128) ||
+        !make_map(&mk, a.k, (uint64_t)a.B * a.Hkv * a.T, D, 128) ||
+        !make_map(&mv, a.v, (uint64_t)a.B * a.Hkv * a.T, D, 128))
         return cudaErrorInvalidValue;
     SdpaParams p;
     p.B = a.B;
@@ -914,6 +886,10 @@ cudaError_t wsum_launch(const StepArgs& a) {
 }
 
 }  // namespace
+
+bool tc_make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows) {
+    return make_map(m, base, rows, d, box_rows);
+}
 
 bool tc_supported(int device, int d) {
     if (d != 64 && d != 128) return false;

@@ -1,6 +1,8 @@
 // tc.h -- tensor-core (tcgen05 / TMEM / TMA) kernels of the bf16 H2O step.
 #pragma once
 
+#include <cuda.h>
+
 #include "kernels.h"
 
 namespace h2o {
@@ -21,5 +23,10 @@ cudaError_t tc_exp2_selftest(const float* x, float* y3, float* y4, float* ym, in
 cudaError_t tc_sdpa(const StepArgs& a);
 // Per-key weight sums added to the scores (writes cand_score / cand_pos).
 cudaError_t tc_wsum(const StepArgs& a);
+// 2-D TMA map over a [rows, d] bf16 matrix: boxes of box_rows rows x 64
+// columns, 128-byte swizzle (the UMMA K-major / MN-major operand layouts).
+bool tc_make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows);
+// Backward of the chunk SDPA on the tensor cores (bf16 inputs; fp32 gradients).
+cudaError_t tc_backward(const BwdArgs& a);
 
 }  // namespace h2o

@@ -322,4 +322,36 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 }  // namespace tc
+
+// ---- role synchronisation shared by the tensor-core kernels -----------------
+// Bounded wait that also gives up once another role has given up.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const WaitBound& wb, int code,
+                                         volatile int* abort_flag) {
+    const uint32_t addr = smem_u32(bar);
+    if (mbar_try_wait(addr, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait_sleep(addr, parity, 20000u)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > wb.ns) {
+            record_error(wb, code);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Every lane waits; the outcome is made warp-uniform so that a give-up never
+// leaves part of a warp behind at a warp-collective instruction.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitBound& wb, int code,
+                                          volatile int* abort_flag) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, wb, code, abort_flag));
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    const uint32_t a = smem_u32(p);
+    return p + (((a + 1023u) & ~1023u) - a);
+}
+
 }  // namespace h2o
