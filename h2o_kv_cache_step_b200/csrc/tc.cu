@@ -460,15 +460,16 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 // ============================================================================
 // Weight sums
 // ============================================================================
-// Persistent: one CTA per SM walks a static list of units (KV group, 128-key
-// block, 1024-row part) in decreasing amount of work. Per unit it holds the
-// key block (the A operand, M = 128 keys) and the part's row table (-log2 LSE
-// per query row, fetched with one bulk copy), and streams 256-row query tiles
-// (the B operand, N = 256): S^T = K Q^T lands in one of two 256-column TMEM
-// buffers, one key per lane. Two consumer warpgroups take alternate tiles;
-// each thread sums its key's weights exp2(s * scale - lse2) over the tile's
-// columns in registers. Each warpgroup writes its own partial per unit; the
-// selection kernel adds all partials of a key in a fixed order.
+// Persistent, two CTAs per SM: each CTA walks a static list of units (KV
+// group, 128-key block, 1024-row part) in decreasing amount of work. Per unit
+// it holds the key block (the A operand, M = 128 keys) and the part's row
+// table (-log2 LSE per query row, fetched with one bulk copy), and streams
+// 128-row query tiles (the B operand, N = 128): S^T = K Q^T lands in one of
+// two 128-column TMEM buffers, one key per lane. One consumer warpgroup of
+// four warps takes the tiles in turn; each thread sums its key's weights
+// exp2(s * scale - lse2) over the tile's columns in registers and writes its
+// key's partial per unit; the selection kernel adds all partials of a key in
+// a fixed order.
 constexpr int kRowsPerUnit = 1024;
 constexpr int kRowTile = 128;
 constexpr int kTilesPerUnit = kRowsPerUnit / kRowTile;
