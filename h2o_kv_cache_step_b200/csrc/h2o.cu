@@ -69,6 +69,9 @@ struct h2o_ctx {
     // log2-domain LSE per flattened group row, [2][groups][bwd_rows_pad]
     float* bwd_rows = nullptr;
     int bwd_rows_pad = 0;
+    // split SDPA workspace (grown on demand when a step splits its units)
+    float* sdpa_part = nullptr;
+    size_t sdpa_part_elems = 0;
     // decode-path workspace (chunks of up to kDecodeMaxT tokens)
     float* dec_part = nullptr;
     float* dec_logits = nullptr;
@@ -344,6 +347,7 @@ int h2o_destroy(h2o_ctx* c) {
     cudaFree(c->Kc);
     cudaFree(c->Vc);
     cudaFree(c->bwd_rows);
+    cudaFree(c->sdpa_part);
     cudaFree(c->ins_K);
     cudaFree(c->ins_V);
     cudaFree(c->ins_slot);
@@ -387,7 +391,9 @@ int h2o_kernel_plan(const h2o_ctx* c, int T, const char** names, int max_names) 
         plan[k++] = "decode_combine_kernel";
         plan[k++] = "decode_wsum_kernel";
     } else if (c->use_tc) {
-        k += tc_kernel_plan(c->B, c->Hq, c->Hkv, c->d, c->C, T, (int)c->n, plan + k, kMaxStepKernels - 2 - k);
+        const int n_eff = insert ? (int)(c->n + T > c->C ? c->C - T : c->n) : (int)c->n;
+        k += tc_kernel_plan(c->B, c->Hq, c->Hkv, c->d, c->C, T, n_eff, c->num_sms, plan + k,
+                            kMaxStepKernels - 2 - k);
     } else {
         plan[k++] = "sdpa_simt_kernel";
         plan[k++] = "wsum_simt_kernel";
@@ -447,6 +453,21 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
     if (decode) {
         H2O_TRY(c, launch_decode(b), "launch decode-path kernels");
     } else if (c->use_tc) {
+        const size_t need = tc_sdpa_part_elems(c->B, c->Hq, c->Hkv, c->d, T, (int)b.n, c->num_sms);
+        if (need > c->sdpa_part_elems) {
+            // the first split step, or one that needs more room: (re)allocate once
+            if (c->sdpa_part) {
+                H2O_TRY(c, cudaStreamSynchronize(s), "sync before SDPA workspace growth");
+                H2O_TRY(c, cudaDeviceSynchronize(), "sync before SDPA workspace growth");
+                cudaFree(c->sdpa_part);
+                c->sdpa_part = nullptr;
+                c->sdpa_part_elems = 0;
+            }
+            H2O_TRY(c, cudaMalloc(&c->sdpa_part, sizeof(float) * need), "cudaMalloc(split SDPA workspace)");
+            c->sdpa_part_elems = need;
+        }
+        b.sdpa_part = c->sdpa_part;
+        b.sdpa_part_elems = c->sdpa_part_elems;
         H2O_TRY(c, tc_sdpa(b), "launch tensor-core SDPA");
         H2O_TRY(c, tc_wsum(b), "launch tensor-core weight sums");
     } else {

@@ -61,6 +61,8 @@ struct StepArgs {
     float* dec_logits;   // decode path: scaled logits [group][row][C + kDecodeMaxT]
     float* dec_lse2;     // decode path: log2-sum-exp per (group, row)
     const void* tmaps;   // device copy of the step's TMA descriptors (tensor-core path)
+    float* sdpa_part;    // split SDPA: partial outputs, maxima and sums (tensor-core path)
+    size_t sdpa_part_elems;
     WaitBound wb;
     cudaStream_t stream;
     int num_sms;

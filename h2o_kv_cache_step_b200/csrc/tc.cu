@@ -32,6 +32,7 @@
 //   (per-CTA partials); the selection kernel adds the parts in a fixed order.
 #include <cuda.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "tc.h"
@@ -111,10 +112,14 @@ struct SdpaParams {
     int nbc;      // cache key blocks = ceil(n / 128)
     int npairs;   // head pairs per KV group = ceil(G / 2)
     int rows_pad; // row stride of nlse2
+    int nsplit;   // pieces the cache blocks of a unit are split into (1: none)
+    int cb_per;   // cache blocks per piece
     float scale_log2;
     __nv_bfloat16* out;
     float* lse;
     float* nlse2;  // [groups][rows_pad]: -(log2-domain LSE) per flattened group row
+    float* part_o;   // nsplit > 1: [nsplit][B*Hq*T][D] unnormalised partial outputs
+    float* part_ml;  // nsplit > 1: [nsplit][B*Hq*T][2] their log2-domain maximum and sum
     WaitBound wb;
 };
 
@@ -143,14 +148,22 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     // unit = (row tile, KV group, head pair); the last row tiles (most keys) first
     const int G = p.Hq / p.Hkv;
     const int per_mblk = p.B * p.Hkv * p.npairs;
-    const int mblk = p.n_mblk - 1 - (int)(blockIdx.x / per_mblk);
-    const int rest = blockIdx.x % per_mblk;
+    const int unit = blockIdx.x / p.nsplit, piece = blockIdx.x % p.nsplit;
+    const int mblk = p.n_mblk - 1 - unit / per_mblk;
+    const int rest = unit % per_mblk;
     const int bg = rest / p.npairs, pr = rest % p.npairs;
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int hA = g * G + 2 * pr;
     const bool hasB = 2 * pr + 1 < G;
     const int m0 = mblk * 128;
-    const int nb = p.nbc + mblk + 1;  // cache blocks, then chunk blocks 0..mblk
+    // this piece's key blocks: cache blocks cb0 .. cb0 + ncb - 1, then (in the
+    // last piece) the chunk blocks 0..mblk; local block jj is global block
+    // gblock(jj) (cache blocks first, then the chunk's)
+    const bool last_piece = piece == p.nsplit - 1;
+    const int cb0 = min(p.nbc, piece * p.cb_per);
+    const int ncb = min(p.nbc, last_piece ? p.nbc : cb0 + p.cb_per) - cb0;
+    const int nb = ncb + (last_piece ? mblk + 1 : 0);
+    auto gblock = [&](int jj) { return jj < ncb ? cb0 + jj : p.nbc + (jj - ncb); };
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -199,7 +212,8 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                                     (b * p.Hq + hA + 1) * p.T + m0, q_full);
             }
             int L = 0;
-            auto load_kv = [&](bool isV, int j) -> bool {
+            auto load_kv = [&](bool isV, int jj) -> bool {
+                const int j = gblock(jj);
                 const int slot = L % RING;
                 if (!wait_bar(ring_empty + slot, ((L / RING) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag))
                     return false;
@@ -332,7 +346,8 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free + X);
             // visible columns of this row in block j: col < limit
-            const int limit = (j < p.nbc) ? p.n - 128 * j : min(i, p.T - 1) - 128 * (j - p.nbc) + 1;
+            const int jg = gblock(j);
+            const int limit = (jg < p.nbc) ? p.n - 128 * jg : min(i, p.T - 1) - 128 * (jg - p.nbc) + 1;
             if (limit < 128) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
@@ -421,7 +436,29 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             m_run = m_use;
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && warp_wait(pv_done + 2 * X + 1, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
+        if (ok && p.nsplit > 1 && warp_wait(pv_done + 2 * X + 1, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
+            // one piece of a split unit: the unnormalised output, its maximum
+            // and its sum, for sdpa_combine_kernel
+            fence_after_sync();
+            const size_t row = (size_t)(b * p.Hq + h) * p.T + i;
+            const size_t rows = (size_t)p.B * p.Hq * p.T;
+            float* prow_o = p.part_o + ((size_t)piece * rows + row) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tc::tmem_ld32(tO + lane_off + 32 * c, o);
+                tc::tmem_ld_wait();
+                if (i < p.T) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        *reinterpret_cast<float4*>(prow_o + 32 * c + 4 * q4) =
+                            make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
+                                        __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
+                }
+            }
+            if (i < p.T)
+                *reinterpret_cast<float2*>(p.part_ml + ((size_t)piece * rows + row) * 2) = make_float2(m_run, l_run);
+        } else if (ok && p.nsplit == 1 && warp_wait(pv_done + 2 * X + 1, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
             fence_after_sync();
             const float inv = 1.f / l_run;
             __nv_bfloat16* orow = p.out + ((size_t)(b * p.Hq + h) * p.T + i) * D;
@@ -454,6 +491,42 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     if (warp == 1) {
         fence_after_sync();
         tc::tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    }
+}
+
+// Merges the pieces of split SDPA units, one warp per query row: with the
+// pieces' log2-domain maxima m_s and sums l_s, M = max m_s,
+// L = sum_s l_s 2^(m_s - M), O = sum_s 2^(m_s - M) O_s / L; writes O (bf16),
+// the natural-log LSE and -log2 LSE per flattened group row.
+template <int D>
+__global__ void __launch_bounds__(256)
+sdpa_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, int nsplit, int Hq,
+                    int Hkv, int T, int tmax, int rows_pad, int rows, __nv_bfloat16* __restrict__ out,
+                    float* __restrict__ lse, float* __restrict__ nlse2) {
+    const int row = (blockIdx.x * blockDim.x + threadIdx.x) / 32, lane = threadIdx.x % 32;
+    if (row >= rows) return;  // warp-uniform
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, part_ml[((size_t)s * rows + row) * 2]);
+    float L = 0.f;
+    float o[D / 32];
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) o[c] = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+        const float2 ml = *reinterpret_cast<const float2*>(part_ml + ((size_t)s * rows + row) * 2);
+        const float w = exp2f(ml.x - M);
+        L = fmaf(ml.y, w, L);
+        const float* po = part_o + ((size_t)s * rows + row) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) o[c] = fmaf(po[lane + 32 * c], w, o[c]);
+    }
+    const float inv = 1.f / L;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) out[(size_t)row * D + lane + 32 * c] = __float2bfloat16_rn(o[c] * inv);
+    if (lane == 0) {
+        const int bh = row / T, i = row % T, G = Hq / Hkv;
+        const float lse2 = M + log2f(L);
+        lse[(size_t)bh * tmax + i] = lse2 * kLn2;
+        nlse2[(size_t)(bh / G) * rows_pad + (size_t)(bh % G) * T + i] = -lse2;
     }
 }
 
@@ -810,6 +883,22 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_ro
 
 int nparts_for(int G, int T) { return (G * T + kRowsPerUnit - 1) / kRowsPerUnit; }
 
+// Pieces the cache blocks of each SDPA unit are split into: only when the
+// units (query tiles x KV groups x head pairs) fill less than half of the SMs
+// and the cache is long enough that each piece keeps at least two blocks.
+int sdpa_split_count(int B, int Hq, int Hkv, int T, int n, int num_sms, int* cb_per = nullptr) {
+    const int units = ((T + 127) / 128) * B * Hkv * ((Hq / Hkv + 1) / 2);
+    const int nbc = (n + 127) / 128;
+    int ns = 1;
+    if (units * 2 <= num_sms && nbc >= 4) ns = std::max(1, std::min({num_sms / units, nbc / 2, 8}));
+    // equal pieces of cb cache blocks (the last one takes the rest and the
+    // chunk's blocks): every piece has at least one block
+    const int cb = (nbc + ns - 1) / ns;
+    if (ns > 1) ns = (nbc + cb - 1) / cb;
+    if (cb_per) *cb_per = cb;
+    return ns;
+}
+
 template <int D>
 cudaError_t sdpa_launch(const StepArgs& a) {
     using Cfg = SdpaCfg<D>;
@@ -838,11 +927,24 @@ cudaError_t sdpa_launch(const StepArgs& a) {
     p.lse = a.lse;
     p.nlse2 = a.nlse2;
     p.wb = a.wb;
-    const int grid = p.n_mblk * a.B * a.Hkv * p.npairs;
+    p.nsplit = sdpa_split_count(a.B, a.Hq, a.Hkv, a.T, a.n, a.num_sms, &p.cb_per);
+    const size_t rows = (size_t)a.B * a.Hq * a.T;
+    p.part_o = a.sdpa_part;
+    p.part_ml = a.sdpa_part ? a.sdpa_part + (size_t)p.nsplit * rows * D : nullptr;
+    if (p.nsplit > 1 && (!a.sdpa_part || a.sdpa_part_elems < (size_t)p.nsplit * rows * (D + 2)))
+        return cudaErrorInvalidValue;
+    const int grid = p.n_mblk * a.B * a.Hkv * p.npairs * p.nsplit;
     cudaError_t e = launch_pdl(sdpa_tc_kernel<D>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, a.stream, mq, mkc,
                                mvc, mk, mv, p);
     if (e != cudaSuccess) return e;
     a.log->done("sdpa_tc_kernel", a.stream);
+    if (p.nsplit > 1) {
+        const int blocks = (int)((rows * 32 + 255) / 256);
+        sdpa_combine_kernel<D><<<blocks, 256, 0, a.stream>>>(p.part_o, p.part_ml, p.nsplit, a.Hq, a.Hkv, a.T, a.tmax,
+                                                             a.rows_pad, (int)rows, p.out, p.lse, p.nlse2);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        a.log->done("sdpa_combine_kernel", a.stream);
+    }
     return cudaGetLastError();
 }
 
@@ -911,10 +1013,17 @@ int tc_rows_pad(int Hq, int Hkv, int tmax) {
 
 int tc_partial_count(int Hq, int Hkv, int T) { return nparts_for(Hq / Hkv, T); }
 
-int tc_kernel_plan(int, int, int, int, int, int, int, const char** names, int max_names) {
-    const char* plan[2] = {"sdpa_tc_kernel", "wsum_tc_kernel"};
-    for (int i = 0; i < 2 && i < max_names; ++i) names[i] = plan[i];
-    return 2;
+int tc_kernel_plan(int B, int Hq, int Hkv, int, int, int T, int n, int num_sms, const char** names, int max_names) {
+    const bool split = sdpa_split_count(B, Hq, Hkv, T, n, num_sms) > 1;
+    const char* plan[3] = {"sdpa_tc_kernel", split ? "sdpa_combine_kernel" : "wsum_tc_kernel", "wsum_tc_kernel"};
+    const int k = split ? 3 : 2;
+    for (int i = 0; i < k && i < max_names; ++i) names[i] = plan[i];
+    return k;
+}
+
+size_t tc_sdpa_part_elems(int B, int Hq, int Hkv, int d, int T, int n, int num_sms) {
+    const int ns = sdpa_split_count(B, Hq, Hkv, T, n, num_sms);
+    return ns > 1 ? (size_t)ns * B * Hq * T * (d + 2) : 0;
 }
 
 cudaError_t tc_exp2_selftest(const float* x, float* y3, float* y4, float* ym, int n, cudaStream_t s) {

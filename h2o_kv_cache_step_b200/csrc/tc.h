@@ -16,7 +16,10 @@ int tc_rows_pad(int Hq, int Hkv, int tmax);
 // Number of weight-sum partials (row parts) a chunk of T tokens produces.
 int tc_partial_count(int Hq, int Hkv, int T);
 // Names of the tensor-core kernels one step launches (returns the count).
-int tc_kernel_plan(int B, int Hq, int Hkv, int d, int C, int T, int n, const char** names, int max_names);
+int tc_kernel_plan(int B, int Hq, int Hkv, int d, int C, int T, int n, int num_sms, const char** names,
+                   int max_names);
+// Floats of the workspace a step's split SDPA needs (0 when it does not split).
+size_t tc_sdpa_part_elems(int B, int Hq, int Hkv, int d, int T, int n, int num_sms);
 // Evaluates the polynomial exp2 (degrees 3 and 4) and ex2.approx on x[0..n).
 cudaError_t tc_exp2_selftest(const float* x, float* y3, float* y4, float* ym, int n, cudaStream_t s);
 // Chunk SDPA: O and per-row LSE.

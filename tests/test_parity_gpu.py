@@ -45,6 +45,8 @@ def test_tiny_fp32_workload_lockstep():
     ("bf16", 128, 1, 4, 2, 100, 300, 3),     # chunk longer than the cache
     ("fp32", 128, 1, 4, 2, 200, 96, 4),
     ("fp32", 64, 2, 2, 1, 130, 33, 6),
+    ("bf16", 128, 1, 8, 2, 1500, 200, 9),    # few units, long cache: SDPA split into 2..6 pieces
+    ("bf16", 64, 1, 8, 1, 1100, 130, 10),    # the same at d = 64, ragged last piece
 ])
 def test_small_shapes_lockstep(dtype, d, B, Hq, Hkv, C, T, chunks):
     wl = synth.Workload("small", dtype, B=B, Hq=Hq, Hkv=Hkv, d=d, C=C, T=T, N=T * chunks,
