@@ -163,9 +163,24 @@ def profiled_traffic(wl, name: str, sched):
     return None
 
 
+def sdpa_pieces(wl, n: int, T: int, num_sms: int = 148) -> int:
+    """Pieces the tensor-core SDPA splits each unit's cache blocks into (the
+    library's rule: only when its units fill less than half of the SMs)."""
+    units = -(-T // 128) * wl.B * wl.Hkv * ((wl.G + 1) // 2)
+    nbc = -(-n // 128)
+    if units * 2 > num_sms or nbc < 4:
+        return 1
+    ns = max(1, min(num_sms // units, nbc // 2, 8))
+    cb = -(-nbc // ns)
+    return -(-nbc // cb)
+
+
 def kernel_work(wl, name: str, n: int, T: int):
     """Algorithmic work of one launch: (amount, unit, bound)."""
     pairs = step_pairs(wl, n, T)
+    if "sdpa_combine" in name:                            # partials in, bf16 rows out
+        rows = wl.B * wl.Hq * T
+        return float(rows * sdpa_pieces(wl, n, T) * (wl.d + 2) * 4 + rows * wl.d * 2), "byte", "hbm"
     if "sdpa" in name:
         return 4.0 * wl.d * pairs, "flop", "tensor"      # QK^T + PV
     if "wsum" in name:
@@ -220,12 +235,16 @@ def run_ours(args, rank, world, local_rank):
     sched = sequence_schedule(wl, insert=args.policy == "insert")
 
     t0 = time.time()
-    chunks = []
+    # the whole sequence resident, chunk after chunk: [n_chunks, B, H, T, d]
+    qs = torch.empty((wl.n_chunks, wl.B, wl.Hq, wl.T, wl.d), dtype=tdt, device=dev)
+    ks = torch.empty((wl.n_chunks, wl.B, wl.Hkv, wl.T, wl.d), dtype=tdt, device=dev)
+    vs = torch.empty_like(ks)
     for c in range(wl.n_chunks):
-        q, k, v = synth.chunk(wl, c)
-        chunks.append(tuple(torch.from_numpy(x).to(dev).to(tdt) for x in (q, k, v)))
+        for dst, x in zip((qs, ks, vs), synth.chunk(wl, c)):
+            dst[c].copy_(torch.from_numpy(x).to(dev).to(tdt))
+    chunks = [(qs[c], ks[c], vs[c]) for c in range(wl.n_chunks)]
     torch.cuda.synchronize()
-    in_bytes = sum(t.numel() * t.element_size() for ch in chunks for t in ch)
+    in_bytes = sum(t.numel() * t.element_size() for t in (qs, ks, vs))
     log(f"[rank {rank}] generated {wl.n_chunks} chunks ({in_bytes / 1e6:.0f} MB resident) "
         f"in {time.time() - t0:.1f}s")
     out = torch.empty_like(chunks[0][0])
@@ -237,10 +256,15 @@ def run_ours(args, rank, world, local_rank):
     plan = cache.kernel_plan(wl.T)
     stream = torch.cuda.current_stream()
 
+    outs = None
+    if args.mode == "prefill":
+        outs = torch.empty_like(qs)
+
     def prefill():
+        # one call for the whole sequence (h2o_prefill): each step's attention
+        # to its own chunk may overlap the previous step's eviction
         cache.reset()
-        for (q, k, v) in chunks:
-            cache.step(q, k, v, out=out)
+        cache.prefill(qs, ks, vs, out=outs)
 
     if args.mode == "chunk":
         # one steady-state chunk step per bench step (for profiler captures):

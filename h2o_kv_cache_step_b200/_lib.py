@@ -40,6 +40,7 @@ SIGNATURES = [
     ("h2o_create_ex", _I, [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_P)]),
     ("h2o_destroy", _I, [_P]),
     ("h2o_step", _I, [_P, _P, _P, _P, _P, _I, _P]),
+    ("h2o_prefill", _I, [_P, _P, _P, _P, _P, _I, _I, _P]),
     ("h2o_step_host", _I, [_P, _P, _P, _P, _P, _I, _P]),
     ("h2o_backward", _I, [_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
     ("h2o_step_host_async", _I, [_P, _P, _P, _P, _P, _I, _P]),

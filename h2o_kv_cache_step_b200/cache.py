@@ -76,6 +76,27 @@ class H2OCache:
                                    _stream_ptr(stream)))
         return out
 
+    def prefill(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """nchunks steps in one call: q [nchunks, B, Hq, T, d], k and v
+        [nchunks, B, Hkv, T, d] (contiguous, on the device); returns the
+        outputs [nchunks, B, Hq, T, d]. Same results as step() per chunk."""
+        if q.dim() != 5:
+            raise ValueError("q: need [nchunks, B, Hq, T, d]")
+        nch, T = q.shape[0], q.shape[3]
+        for name, t, heads in (("q", q, self.Hq), ("k", k, self.Hkv), ("v", v, self.Hkv)):
+            if (t.dtype != self.dtype or not t.is_cuda or not t.is_contiguous()
+                    or tuple(t.shape) != (nch, self.B, heads, T, self.d)):
+                raise ValueError(f"{name}: need contiguous CUDA {self.dtype} of shape "
+                                 f"{(nch, self.B, heads, T, self.d)}, got {t.dtype} {tuple(t.shape)}")
+        if out is None:
+            out = torch.empty_like(q)
+        elif out.dtype != q.dtype or tuple(out.shape) != tuple(q.shape) or not out.is_contiguous():
+            raise ValueError("out: need a contiguous tensor like q")
+        self._check(lib().h2o_prefill(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), T, nch,
+                                      _stream_ptr(stream)))
+        return out
+
     def backward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lse: torch.Tensor,
                  dout: torch.Tensor, stream=None):
         """Gradients of one step's attention for the key set it used, taking the

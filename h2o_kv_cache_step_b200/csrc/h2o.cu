@@ -399,13 +399,17 @@ int h2o_kernel_plan(const h2o_ctx* c, int T, const char** names, int max_names) 
         plan[k++] = "wsum_simt_kernel";
     }
     plan[k++] = insert ? "insert_finish_kernel" : "select_kernel";
-    plan[k++] = "scatter_kernel";
+    if (insert) plan[k++] = "scatter_kernel";
     for (int i = 0; i < k && i < max_names; ++i)
         if (names) names[i] = plan[i];
     return k;
 }
 
-int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T, void* stream) {
+// One step. early: the previous kernel on the stream is this context's own
+// previous step (h2o_prefill), so the tensor-core SDPA may attend to the
+// chunk's own keys while that step's eviction still runs.
+static int step_impl(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T, void* stream,
+                     bool early) {
     int rc = check_ctx(c);
     if (rc != H2O_OK) return rc;
     if (T < 1) return fail(c, H2O_ERR_ARG, "T must be >= 1 (got %d)", T);
@@ -439,6 +443,8 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
     // insert-always: eviction first, then the chunk step over the compact
     // cache of the kept entries (attention and weight sums unchanged)
     const bool insert = c->policy == H2O_POLICY_INSERT_ALWAYS;
+    // profiling puts events between the kernels, which ends the overlap
+    a.early = early && !insert && !decode && c->use_tc && a.log == &local_log;
     const int n_kept = insert ? (int)(c->n + T > c->C ? c->C - T : c->n) : (int)c->n;
     StepArgs b = a;
     if (insert) {
@@ -476,14 +482,33 @@ int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out,
     }
     if (insert) {
         H2O_TRY(c, launch_insert_finish(a, n_kept), "launch insert-always score update");
+        H2O_TRY(c, launch_scatter(a), "launch scatter");
     } else {
-        H2O_TRY(c, launch_select(a), "launch select");
+        H2O_TRY(c, launch_select(a), "launch select and copy");
     }
-    H2O_TRY(c, launch_scatter(a), "launch scatter");
     c->last_T = T;
     c->last_n = n_kept;  // the step's cache candidates (all n, or the kept ones under insert-always)
     c->n = std::min<int64_t>(c->C, c->n + T);
     c->P += T;
+    return H2O_OK;
+}
+
+int h2o_step(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T, void* stream) {
+    return step_impl(c, q, k, v, out, T, stream, false);
+}
+
+int h2o_prefill(h2o_ctx* c, const void* q, const void* k, const void* v, void* out, int T, int nchunks,
+                void* stream) {
+    int rc = check_ctx(c);
+    if (rc != H2O_OK) return rc;
+    if (nchunks < 1 || T < 1) return fail(c, H2O_ERR_ARG, "need nchunks >= 1 and T >= 1 (got %d, %d)", nchunks, T);
+    const size_t elem = c->dtype == H2O_FP32 ? 4 : 2;
+    const size_t qb = (size_t)c->B * c->Hq * T * c->d * elem, kb = (size_t)c->B * c->Hkv * T * c->d * elem;
+    for (int i = 0; i < nchunks; ++i) {
+        rc = step_impl(c, q ? (const char*)q + i * qb : nullptr, k ? (const char*)k + i * kb : nullptr,
+                       v ? (const char*)v + i * kb : nullptr, out ? (char*)out + i * qb : nullptr, T, stream, i > 0);
+        if (rc != H2O_OK) return rc;
+    }
     return H2O_OK;
 }
 

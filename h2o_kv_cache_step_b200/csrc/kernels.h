@@ -34,6 +34,9 @@ struct StepArgs {
     int dtype;        // 0 = bf16, 1 = fp32
     int policy;       // eviction ranking: 0 = H2O score, 1 = score / age
     int tmax;         // capacity (in tokens) of the per-step workspace
+    int early;        // the previous kernel on the stream is this context's
+                      // own step: the SDPA may attend to the chunk's keys
+                      // before that step has finished (tensor-core path)
     const void* q;    // [B,Hq,T,d]
     const void* k;    // [B,Hkv,T,d]
     const void* v;    // [B,Hkv,T,d]
@@ -122,9 +125,9 @@ cudaError_t ensure_smem_limit(void (*kernel)(KArgs...), int bytes) {
 // SIMT kernels (fp32 path; any supported d).
 cudaError_t launch_sdpa_simt(const StepArgs& a);
 cudaError_t launch_wsum_simt(const StepArgs& a);
-// Eviction: per (sequence, KV head) radix select + slot map, then K/V copy.
+// Eviction: per (sequence, KV head) radix select + slot map + K/V copy.
 // Decode path (short chunks): split-K SDPA, combine, weight sums from the
-// kept logits; then launch_select with nparts = 1 and launch_scatter.
+// kept logits; then launch_select with nparts = 1.
 constexpr int kDecodeMaxT = 16;      // longest chunk the decode path takes
 // query rows per KV group (G * T) it takes: the split kernel's dot products
 // run on the CUDA cores, and above this the tensor-core chunk path is faster
@@ -171,6 +174,8 @@ struct BwdArgs {
 };
 cudaError_t launch_bwd_simt(const BwdArgs& a);
 
+// Selection, slot map and the kept tokens' K/V copy (sum and normalized
+// policies); scatter_kernel's wide copy (insert-always).
 cudaError_t launch_select(const StepArgs& a);
 cudaError_t launch_scatter(const StepArgs& a);
 // Sets the message h2o_last_error(NULL) reports on this thread.

@@ -13,8 +13,12 @@
 // Selection runs one CTA per (sequence, KV head): an MSB-first radix select
 // over 64-bit keys (order-preserving score bits : position) finds the C-th
 // largest key; block-wide scans then build the free-slot list and the token
-// to slot map. The key/value copy is a separate wide grid of 16-byte vector
-// copies so that HBM bandwidth, not the handful of selection CTAs, bounds it.
+// to slot map, and the same CTA copies the kept chunk tokens' key and value
+// rows into their slots. Once the cache is full few chunk tokens outlive
+// their own step (a few dozen of 1024 on the bench's workloads), so the copy
+// is small, and keeping it here leaves every other SM to the next step's
+// attention, which starts on its chunk-only key blocks while this kernel runs.
+// (scatter_kernel, a wide grid of the same copies, serves insert-always.)
 #include "kernels.h"
 
 namespace h2o {
@@ -92,7 +96,8 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
               uint8_t* __restrict__ cand_kept, int32_t* __restrict__ token_slot,
               float* __restrict__ scores, int32_t* __restrict__ pos,
               const float* __restrict__ partials, int nparts, int C, int T, int n, int tmax, long long P,
-              int policy) {
+              int policy, const uint4* __restrict__ kin, const uint4* __restrict__ vin, uint4* __restrict__ Kc,
+              uint4* __restrict__ Vc, int row_vecs) {
     __shared__ unsigned int hist[256];
     __shared__ unsigned long long scan_scratch[33];
     __shared__ unsigned long long red_min[32], red_max[32];
@@ -100,8 +105,10 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     __shared__ int sh_hi, sh_krem, sh_done;
     extern __shared__ __align__(16) unsigned char dyn[];
 
-    griddep_wait();  // the weight-sum partials are written
+    // the next kernel may start now: it waits for this one before it reads the
+    // cache or writes anything this kernel reads
     griddep_launch_dependents();
+    griddep_wait();  // the weight-sum partials are written
     const size_t bg = blockIdx.x;
     const int m = n + T;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -345,10 +352,41 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         sc[j] = 0.f;
         ps[j] = -1;
     }
+    __syncthreads();  // the token -> slot map is complete
+
+    // ---- 5. copy the kept tokens' key and value rows into their slots: a
+    // warp takes four tokens at a time, 16 bytes per lane per access, every
+    // load of the four issued before any store
+    const int nwarps = (int)(blockDim.x >> 5);
+    for (int tb = 4 * warp; tb < T; tb += 4 * nwarps) {
+        int sl[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) sl[u] = tb + u < T ? ts[tb + u] : -1;
+        if (sl[0] < 0 && sl[1] < 0 && sl[2] < 0 && sl[3] < 0) continue;  // warp-uniform
+        for (int e0 = 0; e0 < row_vecs; e0 += 32) {
+            const int e = e0 + lane;
+            uint4 kx[4], vx[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (sl[u] >= 0 && e < row_vecs) {
+                    const size_t src = (bg * T + tb + u) * (size_t)row_vecs + e;
+                    kx[u] = kin[src];
+                    vx[u] = vin[src];
+                }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (sl[u] >= 0 && e < row_vecs) {
+                    const size_t dst = (bg * C + sl[u]) * (size_t)row_vecs + e;
+                    Kc[dst] = kx[u];
+                    Vc[dst] = vx[u];
+                }
+        }
+    }
 }
 
 // One warp per chunk token row: copy its key and value rows into the slot
-// chosen for it, 16 bytes per lane per access.
+// chosen for it, 16 bytes per lane per access (insert-always; the other
+// policies copy inside select_kernel).
 __global__ void __launch_bounds__(256)
 scatter_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ Kc,
                uint4* __restrict__ Vc, const int32_t* __restrict__ token_slot, int Hkv, int C, int T,
@@ -385,28 +423,23 @@ __global__ void wait_selftest_kernel(WaitBound wb) {
 
 // The selection and copy kernels are launched with programmatic dependent
 // launch: their CTAs start (and fetch their code) while the previous kernel
-// drains, then wait for it in griddep_wait(). Measured on the bench's prefill:
-// -3% step time; the same for the SDPA and weight-sum launches measured no gain.
+// drains, then wait for it in griddep_wait().
 constexpr bool kEarlyLaunch = true;
 
 cudaError_t launch_select(const StepArgs& a) {
     const int m = a.n + a.T;
     const size_t tail = (((size_t)m + 15) & ~(size_t)15) + (size_t)a.C * 4;  // kept flags + free list
     const size_t with_keys = (size_t)m * 8 + tail;
+    const int row_vecs = a.d * (a.dtype == 1 ? 4 : 2) / 16;
     if (cudaError_t e = ensure_smem_limit(select_kernel<true>, kSelectSmemLimit); e != cudaSuccess) return e;
     if (cudaError_t e = ensure_smem_limit(select_kernel<false>, kSelectSmemLimit); e != cudaSuccess) return e;
-    cudaError_t e;
-    if (with_keys <= (size_t)kSelectSmemLimit) {
-        e = launch_ex(kEarlyLaunch, select_kernel<true>, dim3(a.B * a.Hkv), dim3(kSelThreads), with_keys, a.stream, a.cand_score,
-                       a.cand_pos, a.cand_kept, a.token_slot, a.scores, a.pos, (const float*)a.partials,
-                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P, a.policy);
-    } else if (tail <= (size_t)kSelectSmemLimit) {
-        e = launch_ex(kEarlyLaunch, select_kernel<false>, dim3(a.B * a.Hkv), dim3(kSelThreads), tail, a.stream, a.cand_score,
-                       a.cand_pos, a.cand_kept, a.token_slot, a.scores, a.pos, (const float*)a.partials,
-                       a.nparts, a.C, a.T, a.n, a.tmax, (long long)a.P, a.policy);
-    } else {
-        return cudaErrorInvalidConfiguration;
-    }
+    const bool keys_fit = with_keys <= (size_t)kSelectSmemLimit;
+    if (!keys_fit && tail > (size_t)kSelectSmemLimit) return cudaErrorInvalidConfiguration;
+    cudaError_t e = launch_ex(kEarlyLaunch, keys_fit ? select_kernel<true> : select_kernel<false>, dim3(a.B * a.Hkv),
+                              dim3(kSelThreads), keys_fit ? with_keys : tail, a.stream, a.cand_score, a.cand_pos,
+                              a.cand_kept, a.token_slot, a.scores, a.pos, (const float*)a.partials, a.nparts, a.C,
+                              a.T, a.n, a.tmax, (long long)a.P, a.policy, (const uint4*)a.k, (const uint4*)a.v,
+                              (uint4*)a.Kc, (uint4*)a.Vc, row_vecs);
     if (e != cudaSuccess) return e;
     a.log->done("select_kernel", a.stream);
     return cudaGetLastError();

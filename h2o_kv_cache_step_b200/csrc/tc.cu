@@ -114,6 +114,8 @@ struct SdpaParams {
     int rows_pad; // row stride of nlse2
     int nsplit;   // pieces the cache blocks of a unit are split into (1: none)
     int cb_per;   // cache blocks per piece
+    int early;    // wait for the previous kernel only before the first cache
+                  // block and before the epilogue (see sdpa_tc_kernel)
     float scale_log2;
     __nv_bfloat16* out;
     float* lse;
@@ -156,14 +158,18 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     const int hA = g * G + 2 * pr;
     const bool hasB = 2 * pr + 1 < G;
     const int m0 = mblk * 128;
-    // this piece's key blocks: cache blocks cb0 .. cb0 + ncb - 1, then (in the
-    // last piece) the chunk blocks 0..mblk; local block jj is global block
-    // gblock(jj) (cache blocks first, then the chunk's)
+    // this piece's key blocks: (in the last piece) the chunk blocks 0..mblk
+    // first, then the cache blocks cb0 .. cb0 + ncb - 1; local block jj is
+    // global block gblock(jj) (global numbering: cache blocks, then the
+    // chunk's). The chunk's keys depend only on this step's inputs, so they go
+    // first: in early mode they are attended to while the previous step's
+    // eviction still runs.
     const bool last_piece = piece == p.nsplit - 1;
     const int cb0 = min(p.nbc, piece * p.cb_per);
     const int ncb = min(p.nbc, last_piece ? p.nbc : cb0 + p.cb_per) - cb0;
-    const int nb = ncb + (last_piece ? mblk + 1 : 0);
-    auto gblock = [&](int jj) { return jj < ncb ? cb0 + jj : p.nbc + (jj - ncb); };
+    const int nchk = last_piece ? mblk + 1 : 0;
+    const int nb = nchk + ncb;
+    auto gblock = [&](int jj) { return jj < nchk ? p.nbc + jj : cb0 + (jj - nchk); };
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -190,7 +196,13 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t sbase = smem_u32(smem);
-    griddep_wait();  // inputs written, and the previous step's readers done
+    // Early mode: the step's inputs (q, k, v) were complete before the
+    // previous kernel on the stream started, so only the cache blocks (which
+    // the previous step's eviction rewrites) and the writes of the epilogue
+    // (buffers the previous step reads) wait for it; the loader and the
+    // softmax warps each call griddep_wait() there. Otherwise every thread
+    // waits here.
+    if (!p.early) griddep_wait();  // inputs written, and the previous step's readers done
     griddep_launch_dependents();
 
     if (warp == 0) {
@@ -212,12 +224,17 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                                     (b * p.Hq + hA + 1) * p.T + m0, q_full);
             }
             int L = 0;
+            bool waited = !p.early;
             auto load_kv = [&](bool isV, int jj) -> bool {
                 const int j = gblock(jj);
                 const int slot = L % RING;
                 if (!wait_bar(ring_empty + slot, ((L / RING) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag))
                     return false;
                 const bool cache = j < p.nbc;
+                if (cache && !waited) {
+                    griddep_wait();  // the previous step's eviction has rewritten the cache
+                    waited = true;
+                }
                 const int row = cache ? bg * p.C + 128 * j : bg * p.T + 128 * (j - p.nbc);
                 const CUtensorMap* map = isV ? (cache ? &map_vc : &map_v) : (cache ? &map_kc : &map_k);
                 mbar_arrive_expect_tx(ring_full + slot, Cfg::TILE);
@@ -436,6 +453,7 @@ sdpa_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             m_run = m_use;
         }
         // ------------------------------------------------------------ epilogue
+        if (p.early) griddep_wait();  // the previous step no longer reads out, lse, nlse2
         if (ok && p.nsplit > 1 && warp_wait(pv_done + 2 * X + 1, (nb - 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag)) {
             // one piece of a split unit: the unnormalised output, its maximum
             // and its sum, for sdpa_combine_kernel
@@ -927,6 +945,7 @@ cudaError_t sdpa_launch(const StepArgs& a) {
     p.lse = a.lse;
     p.nlse2 = a.nlse2;
     p.wb = a.wb;
+    p.early = a.early;
     p.nsplit = sdpa_split_count(a.B, a.Hq, a.Hkv, a.T, a.n, a.num_sms, &p.cb_per);
     const size_t rows = (size_t)a.B * a.Hq * a.T;
     p.part_o = a.sdpa_part;
@@ -934,8 +953,12 @@ cudaError_t sdpa_launch(const StepArgs& a) {
     if (p.nsplit > 1 && (!a.sdpa_part || a.sdpa_part_elems < (size_t)p.nsplit * rows * (D + 2)))
         return cudaErrorInvalidValue;
     const int grid = p.n_mblk * a.B * a.Hkv * p.npairs * p.nsplit;
-    cudaError_t e = launch_pdl(sdpa_tc_kernel<D>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, a.stream, mq, mkc,
-                               mvc, mk, mv, p);
+    // early mode: launched as a programmatic dependent of the previous step's
+    // selection, so its CTAs start on the free SMs while that still runs
+    cudaError_t e = a.early ? launch_ex(true, sdpa_tc_kernel<D>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, a.stream,
+                                        mq, mkc, mvc, mk, mv, p)
+                            : launch_pdl(sdpa_tc_kernel<D>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, a.stream,
+                                         mq, mkc, mvc, mk, mv, p);
     if (e != cudaSuccess) return e;
     a.log->done("sdpa_tc_kernel", a.stream);
     if (p.nsplit > 1) {

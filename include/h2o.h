@@ -126,6 +126,19 @@ int h2o_set_policy(h2o_ctx *ctx, int policy);
 int h2o_step(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
              int T, void *stream);
 
+/* nchunks consecutive H2O steps of T tokens each, the same results as that
+ * many h2o_step calls: chunk i is read at q + i * B*Hq*T*d elements (k, v:
+ * + i * B*Hkv*T*d) and its output written at out + i * B*Hq*T*d (device
+ * pointers, layouts as h2o_step, the context's element type). Because every
+ * chunk was written before the call, each step after the first may begin its
+ * attention to the chunk's own tokens while the previous step's eviction is
+ * still running (tensor-core path, H2O_POLICY_SUM and H2O_POLICY_NORMALIZED;
+ * the others run the steps one after another). Stops at the first failing
+ * step and returns its status (the steps before it have been enqueued).
+ * Asynchronous on `stream`. */
+int h2o_prefill(h2o_ctx *ctx, const void *q, const void *k, const void *v, void *out,
+                int T, int nchunks, void *stream);
+
 /* Backward of one step's chunk SDPA with the step's key set held fixed
  * ("Learning how to Forget", paper page, section "Gradient Computation
  * Strategy for Sparse Attention": training through the sparse cache replays
