@@ -89,7 +89,8 @@ constexpr int kFewEvictions = 8;   // up to this many evictions: repeated block 
 constexpr int kPartBatch = 4;      // weight-sum partials loaded per batch
 
 // One CTA per (sequence, KV head). Shared memory: the 64-bit candidate keys
-// (when SMEM_KEYS), the kept flags and the free-slot list.
+// (when SMEM_KEYS), the kept flags, the free-slot list and the kept chunk
+// tokens in position order.
 template <bool SMEM_KEYS>
 __global__ void __launch_bounds__(kSelThreads)
 select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
@@ -119,9 +120,11 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
     float* sc = scores + bg * (size_t)C;
     int32_t* ps = pos + bg * (size_t)C;
     // shared layout: [keys m x 8 B (SMEM_KEYS)] [kept m B] [free list C x 4 B]
+    // [kept tokens T x 4 B]
     unsigned long long* skeys = reinterpret_cast<unsigned long long*>(dyn);
     uint8_t* skept = dyn + (SMEM_KEYS ? (size_t)m * 8 : 0);
     int32_t* sfree = reinterpret_cast<int32_t*>(skept + (((size_t)m + 15) & ~(size_t)15));
+    int32_t* stok = sfree + C;
 
     // ---- 0. candidate scores (old score + weight-sum partials in a fixed
     // part order), positions and keys; every load of a round is issued
@@ -342,6 +345,7 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
             slot = sfree[rt];
             sc[slot] = cs[n + t];
             ps[slot] = (int32_t)(P + t);
+            stok[rt] = t;
         }
         rt += skept[n + t];
         ts[t] = slot;
@@ -352,24 +356,29 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         sc[j] = 0.f;
         ps[j] = -1;
     }
-    __syncthreads();  // the token -> slot map is complete
+    __syncthreads();  // the kept-token list is complete
 
-    // ---- 5. copy the kept tokens' key and value rows into their slots: a
-    // warp takes four tokens at a time, 16 bytes per lane per access, every
-    // load of the four issued before any store
+    // ---- 5. copy the kept tokens' key and value rows into their slots (the
+    // r-th kept token takes free slot r): a warp takes four list entries at a
+    // time, 16 bytes per lane per access, every load of the four issued
+    // before any store
+    const int n_copy = min(n_tok, n_free);
     const int nwarps = (int)(blockDim.x >> 5);
-    for (int tb = 4 * warp; tb < T; tb += 4 * nwarps) {
-        int sl[4];
+    for (int r0 = 4 * warp; r0 < n_copy; r0 += 4 * nwarps) {
+        int tk[4], sl[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) sl[u] = tb + u < T ? ts[tb + u] : -1;
-        if (sl[0] < 0 && sl[1] < 0 && sl[2] < 0 && sl[3] < 0) continue;  // warp-uniform
+        for (int u = 0; u < 4; ++u) {
+            const bool on = r0 + u < n_copy;
+            tk[u] = on ? stok[r0 + u] : 0;
+            sl[u] = on ? sfree[r0 + u] : -1;
+        }
         for (int e0 = 0; e0 < row_vecs; e0 += 32) {
             const int e = e0 + lane;
             uint4 kx[4], vx[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (sl[u] >= 0 && e < row_vecs) {
-                    const size_t src = (bg * T + tb + u) * (size_t)row_vecs + e;
+                    const size_t src = (bg * T + tk[u]) * (size_t)row_vecs + e;
                     kx[u] = kin[src];
                     vx[u] = vin[src];
                 }
@@ -428,7 +437,8 @@ constexpr bool kEarlyLaunch = true;
 
 cudaError_t launch_select(const StepArgs& a) {
     const int m = a.n + a.T;
-    const size_t tail = (((size_t)m + 15) & ~(size_t)15) + (size_t)a.C * 4;  // kept flags + free list
+    // kept flags + free list + kept-token list
+    const size_t tail = (((size_t)m + 15) & ~(size_t)15) + (size_t)a.C * 4 + (size_t)a.T * 4;
     const size_t with_keys = (size_t)m * 8 + tail;
     const int row_vecs = a.d * (a.dtype == 1 ? 4 : 2) / 16;
     if (cudaError_t e = ensure_smem_limit(select_kernel<true>, kSelectSmemLimit); e != cudaSuccess) return e;

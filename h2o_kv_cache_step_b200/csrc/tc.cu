@@ -556,11 +556,12 @@ sdpa_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ 
 // it holds the key block (the A operand, M = 128 keys) and the part's row
 // table (-log2 LSE per query row, fetched with one bulk copy), and streams
 // 128-row query tiles (the B operand, N = 128): S^T = K Q^T lands in one of
-// two 128-column TMEM buffers, one key per lane. One consumer warpgroup of
-// four warps takes the tiles in turn; each thread sums its key's weights
-// exp2(s * scale - lse2) over the tile's columns in registers and writes its
-// key's partial per unit; the selection kernel adds all partials of a key in
-// a fixed order.
+// two 128-column TMEM buffers, one key per lane. Two consumer warpgroups
+// share every tile, one half of its columns each (four consumer warps per SM
+// sub-partition over the two CTAs); each thread sums its key's weights
+// exp2(s * scale - lse2) over its half's columns in registers, the halves
+// meet in shared memory at the end of a unit and the first writes the key's
+// partial; the selection kernel adds all partials of a key in a fixed order.
 constexpr int kRowsPerUnit = 1024;
 constexpr int kRowTile = 128;
 constexpr int kTilesPerUnit = kRowsPerUnit / kRowTile;
@@ -573,12 +574,13 @@ struct WsumCfg {
     static constexpr int OFF_K = 0;                           // key block
     static constexpr int OFF_Q = OFF_K + TILE;                // [QS] query tiles
     static constexpr int OFF_ROW = OFF_Q + QS * TILE;         // [2] row tables (-lse2)
-    static constexpr int OFF_BAR = OFF_ROW + 2 * kRowsPerUnit * 4;
-    static constexpr int NBAR = 16;
+    static constexpr int OFF_RED = OFF_ROW + 2 * kRowsPerUnit * 4;  // [2][128] second half's sums
+    static constexpr int OFF_BAR = OFF_RED + 2 * 128 * 4;
+    static constexpr int NBAR = 24;
     static constexpr int SMEM_RAW = OFF_BAR + NBAR * 8 + 16 + 1024;
     // at least ~80 KB so that no more than two CTAs (2 x 256 TMEM columns) share an SM
     static constexpr int SMEM = SMEM_RAW > 80 * 1024 ? SMEM_RAW : 80 * 1024;
-    static constexpr int THREADS = 192;                       // producer, MMA, 4 consumer warps
+    static constexpr int THREADS = 320;                       // producer, MMA, 8 consumer warps
     static constexpr uint32_t IDESC = tc::idesc_bf16_f32(128, kRowTile, false);
 };
 
@@ -645,6 +647,8 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     uint64_t* s_full = q_empty + QS;    // [2]
     uint64_t* s_empty = s_full + 2;     // [2], 4 arrivals
     uint64_t* drain = s_empty + 2;
+    uint64_t* red_full = drain + 1;     // [2], 4 arrivals: the second half's sums written
+    uint64_t* red_empty = red_full + 2; // [2], 4 arrivals: read by the first half
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -654,9 +658,11 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         mbar_init(k_empty, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(r_full + s, 1);
-            mbar_init(r_empty + s, 4);
+            mbar_init(r_empty + s, 8);
             mbar_init(s_full + s, 1);
-            mbar_init(s_empty + s, 4);
+            mbar_init(s_empty + s, 8);
+            mbar_init(red_full + s, 4);
+            mbar_init(red_empty + s, 4);
         }
         for (int s = 0; s < QS; ++s) {
             mbar_init(q_full + s, 1);
@@ -727,7 +733,9 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         // ----------------------------------------------------------- MMA issuer
         int uc = 0, qc = 0, tc_ = 0;
         bool ok = true;
-        const uint32_t sK = sbase + Cfg::OFF_K;
+        // descriptors: a base value plus constant offsets (start address >> 4)
+        const uint64_t dK = desc_kmajor_sw128(sbase + Cfg::OFF_K);
+        const uint64_t dQ0 = desc_kmajor_sw128(sbase + Cfg::OFF_Q);
         for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++uc) {
             const WsumUnit w = wsum_unit(p, u);
             if (!(ok = warp_wait(k_full, uc & 1, p.wb, kDevTimeoutTmaWait, abort_flag))) break;
@@ -739,12 +747,11 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 if (!ok) break;
                 fence_after_sync();
                 if (lane == 0) {
-                    const uint32_t sQ = sbase + Cfg::OFF_Q + qs * Cfg::TILE;
+                    const uint64_t dQ = dQ0 + (uint64_t)((qs * Cfg::TILE) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-                        tc::mma_bf16_ss(tmem + 128 * sb, desc_kmajor_sw128(sK + off), desc_kmajor_sw128(sQ + off),
-                                        Cfg::IDESC, kk > 0);
+                        const uint64_t off = (uint64_t)(((kk >> 2) * Cfg::HALF + (kk & 3) * 32) >> 4);
+                        tc::mma_bf16_ss(tmem + 128 * sb, dK + off, dQ + off, Cfg::IDESC, kk > 0);
                     }
                     tc::mma_commit(s_full + sb);
                     tc::mma_commit(q_empty + qs);
@@ -765,6 +772,9 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int quad = warp & 3;
         const int kr = quad * 32 + lane;         // key row = TMEM lane
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int half = (warp - 2) >> 2;        // columns 64 * half .. 64 * half + 63 of every tile
+        const int cb = 64 * half;
+        float* red = reinterpret_cast<float*>(smem + Cfg::OFF_RED);
         int uc = 0, tc_ = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++uc) {
@@ -781,68 +791,85 @@ wsum_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 const int tcur = tc_++;
                 if (!(ok = warp_wait(s_full + sb, (tcur >> 1) & 1, p.wb, kDevTimeoutMmaWait, abort_flag))) break;
                 fence_after_sync();
-                float s[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(tmem + 128 * sb + lane_off + 32 * c, v);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(v[e]);
-                }
-                tc::tmem_ld_wait();
-                fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(s_empty + sb);
+                // this half's 64 columns of the tile in two chunks of 32: the
+                // second chunk's TMEM load is in flight while the first is
+                // summed, and the buffer is released as soon as it has landed
+                const uint32_t tS = tmem + 128 * sb + lane_off + cb;
                 const int ncols = min(kRowTile, w.r_end - r0);  // valid rows in the tile
                 const int last = min(r0 + kRowTile - 1, w.r_end - 1);
                 const bool causal = !w.cache && ((last / p.T != r0 / p.T) || (r0 % p.T) < w.t0 + 127);
-                const float4* rt4 = reinterpret_cast<const float4*>(rowt + kRowTile * tt);
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                if (ncols == kRowTile && !causal) {
+                const bool fast = ncols == kRowTile && !causal;
+                const float* rt = rowt + kRowTile * tt;
+                float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+                auto sum_chunk = [&](const uint32_t(&v)[32], int c0) {
+                    if (fast) {
+                        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-                    for (int q4 = 0; q4 < 32; ++q4) {
-                        const float4 L = rt4[q4];
-                        float w0 = fmaf(s[4 * q4 + 0], p.scale_log2, L.x);
-                        float w1 = fmaf(s[4 * q4 + 1], p.scale_log2, L.y);
-                        float w2 = fmaf(s[4 * q4 + 2], p.scale_log2, L.z);
-                        float w3 = fmaf(s[4 * q4 + 3], p.scale_log2, L.w);
-                        if ((q4 & 7) < kPolyPairsOf8Wsum) {
-                            const float2 e01 = tc::exp2_poly3_x2_ftz(make_float2(w0, w1));
-                            const float2 e23 = tc::exp2_poly3_x2_ftz(make_float2(w2, w3));
-                            w0 = e01.x;
-                            w1 = e01.y;
-                            w2 = e23.x;
-                            w3 = e23.y;
-                        } else {
-                            w0 = ex2(w0);
-                            w1 = ex2(w1);
-                            w2 = ex2(w2);
-                            w3 = ex2(w3);
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 Lr = *reinterpret_cast<const float4*>(rt + c0 + 4 * q4);
+                            float2 w01 = tc::ffma2(make_float2(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1])),
+                                                   sc2, make_float2(Lr.x, Lr.y));
+                            float2 w23 = tc::ffma2(make_float2(__uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3])),
+                                                   sc2, make_float2(Lr.z, Lr.w));
+                            if (q4 < kPolyPairsOf8Wsum) {
+                                w01 = tc::exp2_poly3_x2_ftz(w01);
+                                w23 = tc::exp2_poly3_x2_ftz(w23);
+                            } else {
+                                w01 = make_float2(ex2(w01.x), ex2(w01.y));
+                                w23 = make_float2(ex2(w23.x), ex2(w23.y));
+                            }
+                            // flush-to-zero adds: the polynomial exp2 leaves values
+                            // below 2^-126 as subnormals, which must count as 0
+                            a01 = tc::fadd2_ftz(a01, w01);
+                            a23 = tc::fadd2_ftz(a23, w23);
                         }
-                        // flush-to-zero adds: the polynomial exp2 leaves values
-                        // below 2^-126 as subnormals, which must count as 0
-                        a0 = tc::fadd_ftz(a0, w0);
-                        a1 = tc::fadd_ftz(a1, w1);
-                        a2 = tc::fadd_ftz(a2, w2);
-                        a3 = tc::fadd_ftz(a3, w3);
-                    }
-                } else {
-                    // rows past the part's end, or a causal chunk key: row i
-                    // of column c (i advances with c and wraps at the head end)
-                    int i = r0 % p.T;
+                    } else {
+                        // rows past the part's end, or a causal chunk key: row i
+                        // of column c (i advances with c and wraps at the head end)
+                        int i = (r0 + c0) % p.T;
 #pragma unroll
-                    for (int c = 0; c < kRowTile; ++c) {
-                        const float wv = ex2(fmaf(s[c], p.scale_log2, rowt[kRowTile * tt + c]));
-                        const bool vis = (c < ncols) && (i >= t_key);
-                        a0 = tc::fadd_ftz(a0, vis ? wv : 0.f);
-                        if (++i == p.T) i = 0;
+                        for (int e = 0; e < 32; ++e) {
+                            const int c = c0 + e;
+                            const float wv = ex2(fmaf(__uint_as_float(v[e]), p.scale_log2, rt[c]));
+                            const bool vis = (c < ncols) && (i >= t_key);
+                            a01.x = tc::fadd_ftz(a01.x, vis ? wv : 0.f);
+                            if (++i == p.T) i = 0;
+                        }
                     }
-                }
-                acc += (a0 + a1) + (a2 + a3);
+                };
+                uint32_t va[32], vb[32];
+                tc::tmem_ld32(tS, va);
+                tc::tmem_ld_wait();
+                tc::reg_fence(va);
+                tc::tmem_ld32(tS + 32, vb);
+                sum_chunk(va, cb);
+                tc::tmem_ld_wait();
+                tc::reg_fence(vb);
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_empty + sb);
+                sum_chunk(vb, cb + 32);
+                acc += (a01.x + a01.y) + (a23.x + a23.y);
             }
             if (!ok) break;
-            if (kr < w.n_keys)
-                p.partials[((size_t)w.ru * p.groups + w.bg) * (size_t)(p.C + p.tmax) + w.cand0 + kr] = acc;
+            // the two halves' sums of a key meet in shared memory; the first
+            // half adds them (first + second, a fixed order) and writes the
+            // unit's partial
+            float* rs = red + st * 128;
+            if (half == 1) {
+                if (!(ok = warp_wait(red_empty + st, ((uc >> 1) & 1) ^ 1, p.wb, kDevTimeoutSlotWait, abort_flag)))
+                    break;
+                rs[kr] = acc;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(red_full + st);
+            } else {
+                if (!(ok = warp_wait(red_full + st, (uc >> 1) & 1, p.wb, kDevTimeoutSlotWait, abort_flag))) break;
+                const float tot = acc + rs[kr];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(red_empty + st);
+                if (kr < w.n_keys)
+                    p.partials[((size_t)w.ru * p.groups + w.bg) * (size_t)(p.C + p.tmax) + w.cand0 + kr] = tot;
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(r_empty + st);
         }
