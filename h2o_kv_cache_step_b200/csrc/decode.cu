@@ -66,6 +66,7 @@ decode_split_kernel(const E* __restrict__ q, const E* __restrict__ k, const E* _
     const E* ksrc = chunk ? k + (size_t)bg * T * D : Kc + ((size_t)bg * C + j0) * D;
     const E* vsrc = chunk ? v + (size_t)bg * T * D : Vc + ((size_t)bg * C + j0) * D;
     constexpr int V16 = 16 / (int)sizeof(E);  // elements per 16-byte load (rows are 16-byte aligned)
+#pragma unroll 4
     for (int e = threadIdx.x * V16; e < nk * D; e += blockDim.x * V16) {
         const int j = e / D, x = e % D;
         E kv[V16], vv[V16];
@@ -130,9 +131,15 @@ decode_split_kernel(const E* __restrict__ q, const E* __restrict__ k, const E* _
 
 // One CTA per (query row r, group): O = sum_s 2^(m_s - M) O_s / L and the
 // row's log-sum-exp, with M = max_s m_s, L = sum_s 2^(m_s - M) l_s (slices
-// with no visible key have m_s = -inf and add nothing).
+// with no visible key have m_s = -inf and add nothing). Four groups of D
+// threads each merge every fourth slice online (thread x holds column x),
+// twelve slices' loads in flight at a time, and the four results meet in
+// shared memory: a long chain of dependent loads would bound this kernel.
+constexpr int kCombGroups = 4;
+constexpr int kCombBatch = 12;
+
 template <typename E, int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kCombGroups * D)
 decode_combine_kernel(const float* __restrict__ part, E* __restrict__ out, float* __restrict__ lse,
                       float* __restrict__ lse2_rows, int Hq, int Hkv, int T, int nsplit, int tmax) {
     griddep_wait();
@@ -143,40 +150,51 @@ decode_combine_kernel(const float* __restrict__ part, E* __restrict__ out, float
     const int h = g * G + r / T, i = r % T;
     const float* pr = part + ((size_t)bg * nsplit * R + r) * (D + 2);
     const size_t sstride = (size_t)R * (D + 2);
-    extern __shared__ float ssm[];  // [nsplit] slice maxima, [nsplit] sums, [nsplit] weights
-    float* sm = ssm;
-    float* sl = ssm + nsplit;
-    float* sw = ssm + 2 * nsplit;
-    __shared__ float sM, sL;
-    for (int s = threadIdx.x; s < nsplit; s += blockDim.x) {
-        sm[s] = pr[s * sstride + D];
-        sl[s] = pr[s * sstride + D + 1];
+    const int x = threadIdx.x % D, sg = threadIdx.x / D;
+    float M = -INFINITY, L = 0.f, acc = 0.f;
+    for (int s0 = sg; s0 < nsplit; s0 += kCombGroups * kCombBatch) {
+        float ms[kCombBatch], ls[kCombBatch], os[kCombBatch];
+#pragma unroll
+        for (int u = 0; u < kCombBatch; ++u) {
+            const int sl = s0 + kCombGroups * u;
+            const bool on = sl < nsplit;
+            ms[u] = on ? pr[sl * sstride + D] : -INFINITY;
+            ls[u] = on ? pr[sl * sstride + D + 1] : 0.f;
+            os[u] = on ? pr[sl * sstride + x] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kCombBatch; ++u) {
+            if (ms[u] == -INFINITY) continue;
+            const float Mn = fmaxf(M, ms[u]);
+            const float a = exp2f(M - Mn);  // 0 while M is -inf
+            const float w = exp2f(ms[u] - Mn);
+            acc = fmaf(acc, a, w * os[u]);
+            L = fmaf(L, a, w * ls[u]);
+            M = Mn;
+        }
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float M = -INFINITY;
-        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, sm[s]);
-        sM = M;
-    }
-    __syncthreads();
-    const float M = sM;
-    for (int s = threadIdx.x; s < nsplit; s += blockDim.x)
-        sw[s] = (sm[s] == -INFINITY) ? 0.f : exp2f(sm[s] - M);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float L = 0.f;
-        for (int s = 0; s < nsplit; ++s) L = fmaf(sw[s], sl[s], L);
-        sL = L;
-    }
-    const int x = threadIdx.x;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < nsplit; ++s) acc = fmaf(sw[s], pr[s * sstride + x], acc);
-    __syncthreads();
-    const float L = sL;
-    out[(((size_t)b * Hq + h) * T + i) * D + x] = from_f32<E>(acc / L);
+    __shared__ float gM[kCombGroups], gL[kCombGroups];
+    __shared__ float gacc[kCombGroups][D];
+    gacc[sg][x] = acc;
     if (x == 0) {
-        const float l2 = M + log2f(L);
+        gM[sg] = M;
+        gL[sg] = L;
+    }
+    __syncthreads();
+    if (sg != 0) return;
+    float Mt = gM[0];
+#pragma unroll
+    for (int q2 = 1; q2 < kCombGroups; ++q2) Mt = fmaxf(Mt, gM[q2]);
+    float Lt = 0.f, at = 0.f;
+#pragma unroll
+    for (int q2 = 0; q2 < kCombGroups; ++q2) {
+        const float w = gM[q2] == -INFINITY ? 0.f : exp2f(gM[q2] - Mt);
+        Lt = fmaf(w, gL[q2], Lt);
+        at = fmaf(w, gacc[q2][x], at);
+    }
+    out[(((size_t)b * Hq + h) * T + i) * D + x] = from_f32<E>(at / Lt);
+    if (x == 0) {
+        const float l2 = Mt + log2f(Lt);
         lse[((size_t)b * Hq + h) * tmax + i] = l2 * kLn2;
         lse2_rows[(size_t)bg * R + r] = l2;
     }
@@ -196,6 +214,7 @@ decode_wsum_kernel(const float* __restrict__ logits, const float* __restrict__ l
     const float* lr = logits + (size_t)bg * R * lstride + c;
     const float* l2 = lse2_rows + (size_t)bg * R;
     float acc = 0.f;
+#pragma unroll 8
     for (int r = 0; r < R; ++r) acc += exp2f(lr[(size_t)r * lstride] - l2[r]);
     partials[(size_t)bg * cstride + c] = acc;
 }
@@ -216,7 +235,7 @@ cudaError_t launch_decode_typed(const StepArgs& a) {
                               lstride, scale_log2);
     if (e != cudaSuccess) return e;
     a.log->done("decode_split_kernel", a.stream);
-    e = launch_ex(true, decode_combine_kernel<E, D>, dim3(R, groups), dim3(D), sizeof(float) * 3 * nsplit, a.stream,
+    e = launch_ex(true, decode_combine_kernel<E, D>, dim3(R, groups), dim3(kCombGroups * D), 0, a.stream,
                   (const float*)a.dec_part, (E*)a.out, a.lse, a.dec_lse2, a.Hq, a.Hkv, a.T, nsplit, a.tmax);
     if (e != cudaSuccess) return e;
     a.log->done("decode_combine_kernel", a.stream);

@@ -155,6 +155,8 @@ def test_set_policy_rejects_unknown():
     ("fp32", 128, 2, 2, 100, 16, 0),   # T = 16, the longest decode chunk (MHA)
     ("fp32", 64, 4, 2, 130, 3, 0),
     ("bf16", 128, 8, 2, 300, 2, 1),    # normalized policy
+    ("bf16", 128, 8, 2, 4096, 1, 0),   # a long cache: 65 slices per group
+    ("fp32", 64, 4, 2, 2600, 2, 0),    # 42 slices, fp32
 ])
 def test_decode_path_lockstep(dtype, d, Hq, Hkv, C, T, policy):
     """Chunks of T <= 16 tokens take the split-K decode kernels; lockstep
@@ -168,9 +170,10 @@ def test_decode_path_lockstep(dtype, d, Hq, Hkv, C, T, policy):
     for c in range(2):  # cold start
         q, k, v = synth.chunk(wl, c)
         lockstep_full(cache, q, k, v, dtype, wl.C, policy=policy)
-    K, V, S, pos = synth.random_state(wl, n=wl.C, P=1000, seed=T)
+    P0 = max(1000, 2 * wl.C)
+    K, V, S, pos = synth.random_state(wl, n=wl.C, P=P0, seed=T)
     cache.set_state(to_dev(K, dtype), to_dev(V, dtype), torch.from_numpy(S).cuda(),
-                    torch.from_numpy(pos).cuda(), P=1000, n=wl.C)
+                    torch.from_numpy(pos).cuda(), P=P0, n=wl.C)
     for c in range(2, wl.n_chunks):
         q, k, v = synth.chunk(wl, c)
         lockstep_full(cache, q, k, v, dtype, wl.C, policy=policy)
