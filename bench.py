@@ -178,6 +178,15 @@ def sdpa_pieces(wl, n: int, T: int, num_sms: int = 148) -> int:
 def kernel_work(wl, name: str, n: int, T: int):
     """Algorithmic work of one launch: (amount, unit, bound)."""
     pairs = step_pairs(wl, n, T)
+    e = 2 if wl.dtype == "bf16" else 4
+    groups = wl.B * wl.Hkv
+    if name.startswith("decode_"):                        # decode path: bytes each kernel must move
+        R, nsplit = wl.G * T, -(-n // 64) + 1
+        if "split" in name:                               # cache K, V + the chunk's q, k, v once
+            return float(groups * (2 * n * wl.d * e + (R + 2 * T) * wl.d * e)), "byte", "hbm"
+        if "combine" in name:                             # partials in, output rows out
+            return float(groups * R * (nsplit * (wl.d + 2) * 4 + wl.d * e)), "byte", "hbm"
+        return float(groups * R * (n + T) * 4), "byte", "hbm"  # weight sums: the kept logits
     if "sdpa_combine" in name:                            # partials in, bf16 rows out
         rows = wl.B * wl.Hq * T
         return float(rows * sdpa_pieces(wl, n, T) * (wl.d + 2) * 4 + rows * wl.d * 2), "byte", "hbm"
@@ -189,8 +198,6 @@ def kernel_work(wl, name: str, n: int, T: int):
         return 6.0 * wl.d * pairs, "flop", "tensor" if "_tc" in name else "alu"
     if "bwd_dkdv" in name:                                # backward: S, dP recomputed, dV, dK
         return 8.0 * wl.d * pairs, "flop", "tensor" if "_tc" in name else "alu"
-    e = 2 if wl.dtype == "bf16" else 4
-    groups = wl.B * wl.Hkv
     if "select" in name:
         return float(groups * (n + T) * 9 + groups * wl.C * 8), "byte", "hbm"
     if "scatter" in name:
