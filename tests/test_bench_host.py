@@ -58,3 +58,40 @@ def test_profiled_traffic_needs_matching_sources(tmp_path, monkeypatch):
 
 def test_job_throughput_is_all_ranks_over_the_slowest():
     assert bench.job_throughput(65536, 4, 8.0) == pytest.approx(65536 * 4 / 0.008)
+
+
+def test_sdpa_pieces_follow_the_split_rule():
+    """The SDPA splits a unit's cache blocks only when its units fill less than
+    half of the SMs; every piece keeps at least one cache block (the last one
+    also takes the chunk's blocks), and no more CTAs than SMs are launched."""
+    big = synth.WORKLOADS["qwen3-4b-c16384-t512-n128k"]
+    assert bench.sdpa_pieces(WL, WL.C, WL.T) == 1                 # 128 units: no split
+    assert bench.sdpa_pieces(big, big.C, big.T) == 2              # 64 units on 148 SMs
+    assert bench.sdpa_pieces(big, 3 * 128, big.T) == 1            # fewer than 4 cache blocks
+    for wl in synth.WORKLOADS.values():
+        for n in range(0, wl.C + 1, 97):
+            ns = bench.sdpa_pieces(wl, n, wl.T)
+            nbc = -(-n // 128)
+            units = -(-wl.T // 128) * wl.B * wl.Hkv * ((wl.G + 1) // 2)
+            assert 1 <= ns <= 8
+            if ns > 1:
+                assert units * ns <= 148
+                cb = -(-nbc // ns)
+                assert (ns - 1) * cb < nbc                       # the last piece has a cache block too
+
+
+def test_kernel_work_of_the_other_kernels():
+    e = 2  # bf16
+    groups = WL.B * WL.Hkv
+    # the split SDPA's merge reads every piece's fp32 partial row and writes bf16 rows
+    big = synth.WORKLOADS["qwen3-4b-c16384-t512-n128k"]
+    rows = big.B * big.Hq * big.T
+    assert bench.kernel_work(big, "sdpa_combine_kernel", big.C, big.T) == (
+        float(rows * 2 * (big.d + 2) * 4 + rows * big.d * e), "byte", "hbm")
+    # decode: the split kernel reads the cache's K and V once (plus the chunk)
+    b, unit, bound = bench.kernel_work(WL, "decode_split_kernel", WL.C, 1)
+    assert (unit, bound) == ("byte", "hbm")
+    assert b == groups * (2 * WL.C * WL.d * e + (WL.G + 2) * WL.d * e)
+    for name in ("decode_combine_kernel", "decode_wsum_kernel"):
+        assert bench.kernel_work(WL, name, WL.C, 1)[1:] == ("byte", "hbm")
+        assert bench.kernel_work(WL, name, WL.C, 1)[0] > 0
