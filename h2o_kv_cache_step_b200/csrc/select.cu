@@ -174,6 +174,10 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
                 cs[c] = sv[u];
                 cp[c] = pv[u];
             }
+            // a cache slot's stored score becomes its new score now; if the
+            // slot is evicted, placement (phase 4) overwrites it after the
+            // barriers in between (with a chunk token's score, or 0)
+            if (c < n) sc[c] = sv[u];
             const unsigned long long key =
                 ((uint64_t)ordered_bits(rank_value(sv[u], pv[u], policy, P + T)) << 32) | (uint32_t)pv[u];
             if (SMEM_KEYS) skeys[c] = key;
@@ -331,10 +335,8 @@ select_kernel(float* __restrict__ cand_score, int32_t* __restrict__ cand_pos,
         block_exclusive_scan<unsigned long long>((nfree_local << 32) | nk_local, scan_scratch, &total);
     const int n_free = (int)(total >> 32), n_tok = (int)(total & 0xffffffffull);
     int r = (int)(ex >> 32);
-    for (int j = j0; j < j1; ++j) {
+    for (int j = j0; j < j1; ++j)
         if (j >= n || !skept[j]) sfree[r++] = j;
-        else sc[j] = cs[j];  // kept cache slot: its updated score
-    }
     __syncthreads();
 
     // ---- 4. kept chunk tokens, in position order, take the free slots
